@@ -1,0 +1,400 @@
+"""Benchmark of paged-KV long-history prefill attention on B200.
+
+One step = the whole hot path over one synthetic workload: for every piece, pa_prefill (paged
+K/V through the page table, split history) and pa_combine. Default workload: the full
+32,768-token prefill in 2,048-token chunks (16 Q / 2 KV heads, D256, fp16, page size 16),
+the pages' headline shape (BaseRT issue #51: paged vs contiguous KV at 32K).
+
+Prints one JSON line (rank 0): query tokens/s over all GPUs, TFLOP/s, the paged/contiguous
+ratio, the roofline of the prefill kernel, an end-to-end number through host buffers, and the
+fp64 CPU oracle timed on a bounded sample as a baseline. `--impl reference` times the oracle
+alone as the reference arm. Multi-GPU runs are independent replicas (no data exchange).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill-attn query tok/s & TFLOP/s vs BF16 peak; paged/contiguous ratio"
+UNIT = "query tok/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"],
+                    source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    rows.append(f)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                                   default=None)}
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+def oracle_sample_rate(wl, inp, seconds: float, seed: int = 17):
+    """Time the fp64 oracle on a stride sample of (row, head) pairs spread over the whole
+    workload; return (query tok/s estimate, samples, elapsed, threads)."""
+    import numpy as np
+    from oracle import oracle
+    Hq = wl.n_q_heads
+    pieces = wl.pieces
+    total_rows = sum(r for _, r in pieces)
+
+    def run(n):
+        rng = np.random.default_rng(seed)
+        t_sum, pairs = 0.0, 0
+        # stride sample across the workload's query rows, one random head each
+        gidx = np.linspace(0, total_rows - 1, n).astype(np.int64)
+        starts = np.cumsum([0] + [r for _, r in pieces])
+        for i, (h, r) in enumerate(pieces):
+            sel = gidx[(gidx >= starts[i]) & (gidx < starts[i + 1])] - starts[i]
+            if len(sel) == 0:
+                continue
+            heads = rng.integers(0, Hq, size=len(sel)).astype(np.int32)
+            q = inp.piece_q(i)
+            pb = oracle.Problem(q=q, k=inp.k_pool, v=inp.v_pool, hist_len=h, dtype=wl.dtype,
+                                page_table=inp.page_table, scale=wl.scale)
+            t0 = time.perf_counter()
+            oracle.attend(pb, sel, heads)
+            t_sum += time.perf_counter() - t0
+            pairs += len(sel)
+        return t_sum, pairs
+
+    threads = oracle.max_threads()
+    t_cal, p_cal = run(max(8, threads))
+    per_pair = t_cal / max(p_cal, 1)
+    n = int(max(p_cal, min(200000, seconds / max(per_pair, 1e-9))))
+    t, pairs = run(n)
+    # one (row, head) pair is 1/Hq of a query token's attention
+    tok_s = (pairs / Hq) / t
+    return tok_s, pairs, t, threads
+
+
+def reference_arm(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from paged_kv_long_b200.inputs import WORKLOADS, generate
+    wl = WORKLOADS[args.workload]
+    inp = generate(wl, poison=False)
+    steps, warmup = args.steps, args.warmup
+    per_step = max(2.0, min(10.0, 150.0 / max(steps + warmup, 1)))
+    for _ in range(warmup):
+        oracle_sample_rate(wl, inp, per_step / 4)
+    rates, times, cores, pairs = [], [], 1, 0
+    for k in range(steps):
+        r, pairs, t, cores = oracle_sample_rate(wl, inp, per_step, seed=100 + k)
+        rates.append(r)
+        times.append(t)
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": wl.query_rows / value * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "seq_len": wl.total_keys, "pieces": len(wl.pieces),
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{pairs} (row, head) pairs per step, stride-sampled over the "
+                                   f"workload's {wl.query_rows} query rows; ~{per_step:.0f} s per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def time_steps(dw, steps, warmup, flush, stream, record_kernels=False):
+    """Per-step CUDA-event timing with an L2 flush between steps (outside the timed events).
+    Returns (per-step ms list, prefill-kernel ms list per step)."""
+    import torch
+    from paged_kv_long_b200 import binding
+    for _ in range(warmup):
+        flush.zero_()
+        dw.run(stream)
+    torch.cuda.synchronize()
+    step_ms, kern_ms = [], []
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        kev = []
+        e0.record(stream)
+        for i in range(len(dw.wl.pieces)):
+            if record_kernels:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                q, k, v, tab = dw.piece_inputs(i)
+                binding.prefill(dw.plans[i], q, k, v, tab, dw.outs[i], dw.ws, stream)
+                b.record(stream)
+                binding.combine(dw.plans[i], dw.ws, dw.outs[i], stream)
+                kev.append((a, b))
+            else:
+                dw.run_piece(i, stream)
+        e1.record(stream)
+        evs.append((e0, e1, kev))
+    torch.cuda.synchronize()
+    for e0, e1, kev in evs:
+        step_ms.append(e0.elapsed_time(e1))
+        kern_ms.append([a.elapsed_time(b) for a, b in kev])
+    return step_ms, kern_ms
+
+
+def e2e_steps(inp, dw, steps, stream):
+    """End to end through the public API: pinned host inputs -> device, prefill + combine for
+    every piece, outputs -> pinned host, every step. Returns (per-step ms, h2d, d2h bytes)."""
+    import numpy as np
+    import torch
+    wl = inp.wl
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+
+    def pinned(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if dt is not None:
+            t = t.view(torch.int16).view(dt)
+        return t.pin_memory()
+
+    hq = pinned(inp.q.view(np.int16), tdt)
+    hk = pinned(inp.k_pool.view(np.int16), tdt)
+    hv = pinned(inp.v_pool.view(np.int16), tdt)
+    ht = pinned(inp.page_table)
+    houts = [torch.empty(tuple(o.shape), dtype=torch.float32).pin_memory() for o in dw.outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ht))
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+    ms = []
+    with torch.cuda.stream(stream):
+        for k in range(steps + 1):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dw.q.copy_(hq, non_blocking=True)
+            dw.k.copy_(hk, non_blocking=True)
+            dw.v.copy_(hv, non_blocking=True)
+            dw.table.copy_(ht, non_blocking=True)
+            dw.run(stream)
+            for o, ho in zip(dw.outs, houts):
+                ho.copy_(o, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if k > 0:  # the first is a warm-up
+                ms.append(e0.elapsed_time(e1))
+    return ms, h2d, d2h
+
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_long_b200.inputs import WORKLOADS, generate
+    from paged_kv_long_b200.runner import DeviceWorkload
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = WORKLOADS[args.workload]
+    inp = generate(wl, poison=False)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(dev)
+    split_arg = args.splits if args.splits is not None else None
+    dw = DeviceWorkload(inp, dev, paged=True, splits=split_arg, policy=args.policy)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- timed region: K steps of the paged path
+    barrier()
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        step_ms, kern_ms = time_steps(dw, args.steps, args.warmup, flush, stream, record_kernels=True)
+        barrier()
+        wall = time.perf_counter() - wall0
+    clocks = clk.summary()
+    t_step = sum(step_ms) / len(step_ms)
+    if world > 1:
+        tt = torch.tensor([t_step], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step = float(tt.item())
+    tokens = wl.query_rows
+    value = world * tokens / (t_step / 1e3)
+    flops = wl.flops()
+    tflops = flops / (t_step / 1e3) / 1e12
+
+    # ---- prefill kernel roofline: algorithmic FLOPs over its summed launch durations
+    kern_total_ms = sum(sum(k) for k in kern_ms) / len(kern_ms)
+    kern_tflops = flops / (kern_total_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
+
+    # ---- contiguous control at the same split counts (the ratio's denominator)
+    dwc = DeviceWorkload(inp, dev, paged=False, splits=None, policy=args.policy)
+    for i, p in enumerate(dw.plans):   # same S per piece as the paged run
+        from paged_kv_long_b200 import binding
+        h, r = wl.pieces[i]
+        dwc.plans[i] = binding.plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size, r, h,
+                                    wl.dtype, wl.scale, p.splits, "makespan", False)
+    c_ms, c_kern = time_steps(dwc, max(3, args.steps // 2), args.warmup, flush, stream,
+                              record_kernels=True)
+    t_contig = sum(c_ms) / len(c_ms)
+    last_paged = statistics.median(k[-1] for k in kern_ms)
+    last_contig = statistics.median(k[-1] for k in c_kern)
+    del dwc
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = e2e_steps(inp, dw, max(2, min(args.steps, 5)), stream)
+        t_e = sum(e_ms) / len(e_ms)
+        e2e = {"value": world * tokens / (t_e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": t_e}
+
+    launches = args.steps * sum(1 + (1 if p.splits > 1 else 0) for p in dw.plans)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r, pairs, t, cores = oracle_sample_rate(wl, inp, args.cpu_seconds)
+        cpu = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{pairs} (row, head) pairs stride-sampled over all {wl.query_rows} query "
+                         f"rows of the workload, {t:.1f} s of fp64 CPU work, scaled to tok/s"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "seq_len": wl.total_keys, "chunk_rows": wl.pieces[0][1],
+                   "pieces": len(wl.pieces), "n_q_heads": wl.n_q_heads,
+                   "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
+                   "page_size": wl.page_size, "kv_layout": "paged",
+                   "splits": [p.splits for p in dw.plans], "split_policy": args.policy,
+                   "l2": "flushed between steps (512 MiB write outside the timed events)",
+                   "parallelism": f"replicas x{world}"},
+        "tflops": tflops,
+        "paged_contiguous_ratio": t_contig / t_step,
+        "paged_contiguous_ratio_last_chunk": last_contig / last_paged,
+        "contiguous_ms_per_step": t_contig,
+        "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                     "step_frac_of_roofline": t_roof / (t_step / 1e3),
+                     "kernel": "prefill_kernel (pa_prefill)",
+                     "algorithmic_flops_per_step": flops},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c5", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--splits", type=int, default=None,
+                    help="split count for every piece (default: the workload's, else the planner)")
+    ap.add_argument("--policy", default="makespan", choices=["makespan", "cores", "legacy"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+    return gpu_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

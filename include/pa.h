@@ -1,0 +1,180 @@
+/*
+ * pa.h — C ABI of libpa: causal GQA prefill attention of a query chunk against a long
+ * history held in a paged KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (what the pages describe; they give no formula, this is the plain reading):
+ *   "Metal: paged-KV prefill is 4.43x slower than contiguous KV at 32K" (BaseRT issue #51),
+ *   sections "Results" and "Scaling characteristic": prefill attention of a chunk whose
+ *   K/V are read through a paged cache, which must cost about what a contiguous cache costs.
+ *   "perf: scale prefill attention splits with GPU cores on Apple7/8" (splash PR #33),
+ *   section "What changed": the history of a piece is cut into splits so that short pieces
+ *   at long history fill the GPU; a reduce merges the split partials; the planner picks the
+ *   split count and workspace from the core count, KV heads and piece tiles.
+ *
+ *   For chunk row i (absolute position H+i) and Q head h, with G = Hq/Hkv and g = floor(h/G):
+ *     key j (0 <= j <= H+i) is  k_pool[page_table[j / PS]][j % PS][g][:]  (v likewise)
+ *     out[i][h][:] = sum_j softmax_j(scale * q[i][h][:] . K[j][:]) * V[j][:]
+ *   with scale = 1/sqrt(D) unless given. The chunk's own K/V (positions H..H+R-1) must
+ *   already be in the cache.
+ *
+ * Threading and memory: every function is reentrant. The library never allocates, frees or
+ * synchronises device memory in pa_prefill / pa_combine; the caller owns every buffer. All
+ * device work is enqueued on the caller's stream (a cudaStream_t passed as pa_stream_t).
+ * Status codes are returned; nothing throws across the ABI.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same representation as cudaStream_t / CUstream (NULL = the legacy default stream). */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, inconsistent sizes, plan mismatch */
+  PA_ERR_UNSUPPORTED = -2,  /* shape outside the supported set (see pa_plan) */
+  PA_ERR_WORKSPACE = -3,    /* lse_ws missing or smaller than plan->ws_bytes */
+  PA_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
+  PA_ERR_TIMEOUT = -5,      /* a kernel wait gave up (reported by pa_device_error) */
+  PA_ERR_PAGE_INDEX = -6    /* a page-table entry was outside [0, num_pages) */
+} pa_status;
+
+/* Split policies for pa_plan (how the history of a piece is partitioned). */
+typedef enum {
+  /* B200: the split count that minimises the simulated makespan of the launch on
+   * num_sms SMs (units are dispatched longest first), plus the combine's HBM cost. */
+  PA_POLICY_MAKESPAN = 0,
+  /* The rule of splash PR #33 ("What changed"): min(256, max(32, 32*cores/kv_heads)) /
+   * tiles, clamped to 1..32, with cores = num_sms and tiles = Q tiles per KV head. */
+  PA_POLICY_CORES = 1,
+  /* The earlier rule quoted in splash PR #33: clamp(32 / tiles, 1, 32), with tiles taken as
+   * the threadgroups over all KV heads (the reading under which every listed piece got 1). */
+  PA_POLICY_LEGACY = 2
+} pa_policy;
+
+/* Rows of the packed (token, head) Q tile, and keys per KV tile, of the kernel. */
+#define PA_TILE_ROWS 128
+#define PA_TILE_KEYS 128
+#define PA_MAX_SPLITS 32
+
+/*
+ * A launch plan. Filled by pa_plan; callers read it and pass it back unchanged.
+ *
+ * Q rows are packed as (token, head-in-group) pairs with the head index fastest: packed row
+ * r of KV head g is token r / G, Q head g*G + r % G. A Q tile is PA_TILE_ROWS consecutive
+ * packed rows (a tile may start inside a token's head group). Work units are
+ * (KV head, Q tile, split); split s of a tile whose tokens end at t_last covers KV tiles
+ * [s*n/S, (s+1)*n/S) of the n = ceil((H + t_last + 1) / PA_TILE_KEYS) tiles it sees.
+ */
+typedef struct {
+  int32_t num_sms;        /* SMs the plan was made for */
+  int32_t n_q_heads;      /* Hq */
+  int32_t n_kv_heads;     /* Hkv (Hq % Hkv == 0) */
+  int32_t head_dim;       /* D: 64, 128 or 256 */
+  int32_t page_size;      /* PS: power of two, 16..128 (ignored when paged == 0) */
+  int32_t group;          /* G = Hq / Hkv */
+  int32_t chunk_rows;     /* R: query rows of the piece (>= 1) */
+  int32_t q_tiles;        /* ceil(R * G / PA_TILE_ROWS) per KV head */
+  int32_t splits;         /* S: 1..PA_MAX_SPLITS */
+  int32_t paged;          /* 1: k/v are page pools read through page_table; 0: contiguous */
+  int32_t dtype;          /* pa_dtype of q, k, v */
+  int32_t policy;         /* pa_policy used (or -1 when splits was overridden) */
+  int64_t hist_len;       /* H: keys in the cache before the piece */
+  int64_t units;          /* Hkv * q_tiles * S CTAs of the prefill kernel */
+  float scale;            /* softmax scale actually used */
+  float est_us;           /* the planner's time estimate for prefill + combine (microseconds) */
+  uint64_t ws_bytes;      /* bytes of lse_ws needed: S*R*Hq*(D+1)*4 if S > 1, else 0 */
+} pa_plan_t;
+
+/*
+ * pa_plan — choose the split count and workspace for one piece.
+ *   num_sms          SMs of the device (148 on B200); > 0.
+ *   n_q_heads, n_kv_heads, head_dim, page_size, chunk_rows, hist_len, dtype: the piece.
+ *   scale            softmax scale; 0 selects 1/sqrt(head_dim).
+ *   splits_override  0: the policy decides; 1..32: use exactly this split count.
+ *   policy           a pa_policy (used when splits_override == 0).
+ *   paged            1: K/V through a page table; 0: contiguous [H+R][Hkv][D].
+ *   plan             out: the plan (host memory owned by the caller).
+ * Returns PA_OK, PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED. Pure host code; no CUDA calls.
+ * Source: splash PR #33 "What changed" (split count from cores, KV heads and tiles; the
+ * workspace is sized by the planner).
+ */
+int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_size,
+            int chunk_rows, int64_t hist_len, int dtype, float scale, int splits_override,
+            int policy, int paged, pa_plan_t* plan);
+
+/*
+ * pa_prefill — split-KV prefill attention of one piece, enqueued on `stream`.
+ *   q            device, [R][Hq][D] of dtype, contiguous, 16-byte aligned.
+ *   k_pool,v_pool device, paged: [num_pages][PS][Hkv][D]; contiguous: [H+R][Hkv][D]; dtype,
+ *                contiguous, 16-byte aligned. Pool slots that hold no key may hold any bits
+ *                (NaN included); they never reach the output.
+ *   page_table   device int32 [ceil((H+R)/PS)]: logical page -> physical page (paged only;
+ *                may be NULL when paged == 0). An entry outside [0, num_pages) reads zeros
+ *                and raises PA_ERR_PAGE_INDEX in pa_device_error.
+ *   num_pages    pages in each pool (paged only).
+ *   hist_len, chunk_rows: must equal the plan's.
+ *   out          device fp32 [R][Hq][D]. Written when plan->splits == 1.
+ *   lse_ws       device fp32 workspace of ws_bytes >= plan->ws_bytes (used when S > 1):
+ *                partial outputs O_s [S][R][Hq][D] (each normalised over its split), then
+ *                base-2 log-sum-exp of the scaled scores lse_s [S][R][Hq] (-inf: no key).
+ * When S > 1, call pa_combine afterwards on the same stream to produce `out`.
+ * Returns PA_OK or an error status; launch errors are PA_ERR_CUDA. Device-side conditions
+ * (bad page entry, wait timeout) are reported by pa_device_error.
+ */
+int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_pool, const void* v_pool,
+               const int32_t* page_table, int64_t num_pages, int64_t hist_len, int chunk_rows,
+               float* out, float* lse_ws, uint64_t ws_bytes, pa_stream_t stream);
+
+/*
+ * pa_combine — log-sum-exp merge of the S split partials in lse_ws into out (fp32
+ * [R][Hq][D]): out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s.
+ * No-op returning PA_OK when plan->splits == 1. Source: splash PR #33, the prefill
+ * attention "reduce" that merges the split partials (decode-profile tables).
+ */
+int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes, float* out,
+               pa_stream_t stream);
+
+/*
+ * pa_device_error — synchronise the current device, then read (and with reset != 0,
+ * clear) the library's device-side error word. *flags receives its bits
+ * (1: page index out of range, 2: a wait timed out). Returns PA_OK when no bit is set,
+ * PA_ERR_PAGE_INDEX or PA_ERR_TIMEOUT for the first set bit, PA_ERR_CUDA on failure.
+ */
+int pa_device_error(int* flags, int reset);
+
+/* pa_set_wait_timeout_ns — upper bound of every kernel-side wait (default 2e9 ns). A wait
+ * that exceeds it makes the kernel set the timeout bit, stop its work and exit. */
+void pa_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * pa_selftest_timeout — enqueue a one-warp kernel that waits on a barrier nothing ever
+ * completes, with a wait limit of timeout_ns; the wait gives up, sets the timeout bit and
+ * the kernel exits. Lets tests check the timeout path without hanging a GPU.
+ */
+int pa_selftest_timeout(uint64_t timeout_ns, pa_stream_t stream);
+
+/* pa_status_string — static description of a status code. */
+const char* pa_status_string(int status);
+
+/* pa_cores_policy_splits — the split rule of splash PR #33 ("What changed") for a GPU with
+ * `cores` cores, `kv_heads` KV heads and `tiles` tiles per KV head. Pure host function. */
+int pa_cores_policy_splits(int cores, int kv_heads, int tiles);
+
+/* pa_legacy_policy_splits — the earlier rule clamp(32 / tiles, 1, 32) quoted there, with
+ * tiles = threadgroups over all KV heads. Pure host function. */
+int pa_legacy_policy_splits(int kv_heads, int tiles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,218 @@
+"""ctypes binding of ``libpa.so`` — argument marshalling only.
+
+Every step of the attention runs in the library's CUDA kernels; this module checks the
+torch tensors it is given (device, dtype, shape, contiguity) and passes their device pointers
+and the caller's current CUDA stream across the C ABI declared in ``include/pa.h``. There is
+no CPU fallback: if the library is missing or a tensor is not on a CUDA device, it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(PKG, "libpa.so")
+
+PA_F16, PA_BF16 = 0, 1
+POLICIES = {"makespan": 0, "cores": 1, "legacy": 2}
+STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
+          -4: "PA_ERR_CUDA", -5: "PA_ERR_TIMEOUT", -6: "PA_ERR_PAGE_INDEX"}
+EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_device_error", "pa_set_wait_timeout_ns",
+            "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
+            "pa_legacy_policy_splits")
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Plan(ctypes.Structure):
+    """Mirror of ``pa_plan_t``."""
+    _fields_ = [
+        ("num_sms", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("group", ctypes.c_int32),
+        ("chunk_rows", ctypes.c_int32), ("q_tiles", ctypes.c_int32), ("splits", ctypes.c_int32),
+        ("paged", ctypes.c_int32), ("dtype", ctypes.c_int32), ("policy", ctypes.c_int32),
+        ("hist_len", ctypes.c_int64), ("units", ctypes.c_int64), ("scale", ctypes.c_float),
+        ("est_us", ctypes.c_float), ("ws_bytes", ctypes.c_uint64),
+    ]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libpa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libpa.so not built at {p}: run `python -m paged_kv_long_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i32, i64, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
+    lib.pa_plan.argtypes = [i32, i32, i32, i32, i32, i32, i64, i32, ctypes.c_float, i32, i32, i32,
+                            ctypes.POINTER(Plan)]
+    lib.pa_plan.restype = i32
+    lib.pa_prefill.argtypes = [ctypes.POINTER(Plan), vp, vp, vp, vp, i64, i64, i32, vp, vp, u64, vp]
+    lib.pa_prefill.restype = i32
+    lib.pa_combine.argtypes = [ctypes.POINTER(Plan), vp, u64, vp, vp]
+    lib.pa_combine.restype = i32
+    lib.pa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), i32]
+    lib.pa_device_error.restype = i32
+    lib.pa_set_wait_timeout_ns.argtypes = [u64]
+    lib.pa_set_wait_timeout_ns.restype = None
+    lib.pa_selftest_timeout.argtypes = [u64, vp]
+    lib.pa_selftest_timeout.restype = i32
+    lib.pa_status_string.argtypes = [i32]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_cores_policy_splits.argtypes = [i32, i32, i32]
+    lib.pa_cores_policy_splits.restype = i32
+    lib.pa_legacy_policy_splits.argtypes = [i32, i32]
+    lib.pa_legacy_policy_splits.restype = i32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise PaError(status, where)
+
+
+def _dtype_code(dtype) -> int:
+    import torch
+    if dtype in ("f16", torch.float16):
+        return PA_F16
+    if dtype in ("bf16", torch.bfloat16):
+        return PA_BF16
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def plan(n_q_heads: int, n_kv_heads: int, head_dim: int, page_size: int, chunk_rows: int,
+         hist_len: int, dtype="bf16", scale: float = 0.0, splits: int = 0,
+         policy: str = "makespan", paged: bool = True, num_sms: int | None = None) -> Plan:
+    """pa_plan: split count and workspace for one piece (host only)."""
+    if num_sms is None:
+        import torch
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    p = Plan()
+    st = load_library().pa_plan(num_sms, n_q_heads, n_kv_heads, head_dim, page_size, chunk_rows,
+                                hist_len, _dtype_code(dtype), scale, splits, POLICIES[policy],
+                                1 if paged else 0, ctypes.byref(p))
+    _check(st, "pa_plan")
+    return p
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _require_cuda(t, name, dtype=None, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _torch_dtype(p: Plan):
+    import torch
+    return torch.bfloat16 if p.dtype == PA_BF16 else torch.float16
+
+
+def workspace(p: Plan, device=None):
+    """A workspace tensor of plan.ws_bytes (fp32), or None when no split is used."""
+    import torch
+    if p.ws_bytes == 0:
+        return None
+    return torch.empty(p.ws_bytes // 4, dtype=torch.float32, device=device or "cuda")
+
+
+def prefill(p: Plan, q, k_pool, v_pool, page_table, out, ws=None, stream=None):
+    """pa_prefill on torch tensors (see include/pa.h for layouts)."""
+    import torch
+    dt = _torch_dtype(p)
+    R, Hq, Hkv, D = p.chunk_rows, p.n_q_heads, p.n_kv_heads, p.head_dim
+    _require_cuda(q, "q", dt, (R, Hq, D))
+    _require_cuda(k_pool, "k_pool", dt)
+    _require_cuda(v_pool, "v_pool", dt, tuple(k_pool.shape))
+    if p.paged:
+        if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (p.page_size, Hkv, D):
+            raise ValueError("k_pool must be [num_pages, page_size, Hkv, D]")
+        _require_cuda(page_table, "page_table", torch.int32)
+        if page_table.numel() < math.ceil((p.hist_len + R) / p.page_size):
+            raise ValueError("page_table is shorter than ceil((H+R)/page_size)")
+        num_pages, tab = k_pool.shape[0], page_table.data_ptr()
+    else:
+        if k_pool.dim() != 3 or tuple(k_pool.shape) != (p.hist_len + R, Hkv, D):
+            raise ValueError("contiguous k/v must be [H+R, Hkv, D]")
+        num_pages, tab = 0, None
+    out_ptr, ws_ptr, ws_bytes = None, None, 0
+    if p.splits == 1:
+        _require_cuda(out, "out", torch.float32, (R, Hq, D))
+        out_ptr = out.data_ptr()
+    else:
+        _require_cuda(ws, "ws", torch.float32)
+        ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * 4
+    st = load_library().pa_prefill(ctypes.byref(p), q.data_ptr(), k_pool.data_ptr(),
+                                   v_pool.data_ptr(), tab, num_pages, p.hist_len, R, out_ptr,
+                                   ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(st, "pa_prefill")
+
+
+def combine(p: Plan, ws, out, stream=None):
+    """pa_combine: merge split partials into out (no-op when splits == 1)."""
+    import torch
+    if p.splits == 1:
+        return
+    _require_cuda(ws, "ws", torch.float32)
+    _require_cuda(out, "out", torch.float32, (p.chunk_rows, p.n_q_heads, p.head_dim))
+    st = load_library().pa_combine(ctypes.byref(p), ws.data_ptr(), ws.numel() * 4, out.data_ptr(),
+                                   _stream_ptr(stream))
+    _check(st, "pa_combine")
+
+
+def prefill_combine(p: Plan, q, k_pool, v_pool, page_table, out=None, ws=None, stream=None):
+    """pa_prefill followed by pa_combine; allocates out / ws with torch when not given."""
+    import torch
+    if out is None:
+        out = torch.empty((p.chunk_rows, p.n_q_heads, p.head_dim), dtype=torch.float32,
+                          device=q.device)
+    if p.splits > 1 and ws is None:
+        ws = workspace(p, q.device)
+    prefill(p, q, k_pool, v_pool, page_table, out, ws, stream)
+    combine(p, ws, out, stream)
+    return out
+
+
+def device_error(reset: bool = True) -> tuple[int, int]:
+    """(status, flags) of the library's device-side error word (synchronises the device)."""
+    flags = ctypes.c_int(0)
+    st = load_library().pa_device_error(ctypes.byref(flags), 1 if reset else 0)
+    return st, flags.value
+
+
+def set_wait_timeout_ns(ns: int):
+    load_library().pa_set_wait_timeout_ns(ns)
+
+
+def selftest_timeout(timeout_ns: int, stream=None):
+    _check(load_library().pa_selftest_timeout(timeout_ns, _stream_ptr(stream)), "pa_selftest_timeout")

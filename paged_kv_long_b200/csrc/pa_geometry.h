@@ -1,0 +1,58 @@
+// pa_geometry.h — the work decomposition shared by the planner (host) and the kernels
+// (device): packed GQA Q tiles, the keys each tile sees, and the split of those keys.
+//
+// Source of the decomposition: splash PR #33 ("What changed"): a piece is cut into Q tiles,
+// tiles x KV heads x splits are the dispatched units, and the splits partition the history.
+// The packing of (token, head) rows is a B200 choice: one 128-row tensor-core tile holds the
+// G query heads that share a KV head, so each K/V tile is read once for all of them.
+#pragma once
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define PA_HD __host__ __device__ __forceinline__
+#else
+#define PA_HD inline
+#endif
+
+namespace pa {
+
+constexpr int kTileRows = 128;   // packed (token, head) rows per Q tile = tensor-core M
+constexpr int kTileKeys = 128;   // keys per KV tile = tensor-core N of QK^T, K of PV
+constexpr int kMaxSplits = 32;
+
+PA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Q tiles per KV head for R rows and G heads per KV head.
+PA_HD int64_t q_tiles_for(int64_t R, int G) { return ceil_div64(R * G, kTileRows); }
+
+// Last token (chunk-relative, inclusive) held by Q tile qt.
+PA_HD int64_t tile_last_token(int64_t qt, int64_t R, int G) {
+  const int64_t t = (qt * kTileRows + kTileRows - 1) / G;
+  return t < R - 1 ? t : R - 1;
+}
+
+// First token held by Q tile qt.
+PA_HD int64_t tile_first_token(int64_t qt, int G) { return (qt * kTileRows) / G; }
+
+// KV tiles visible to Q tile qt: keys [0, H + t_last + 1).
+PA_HD int64_t tile_kv_tiles(int64_t qt, int64_t R, int G, int64_t H) {
+  return ceil_div64(H + tile_last_token(qt, R, G) + 1, kTileKeys);
+}
+
+// KV tiles [*kt0, *kt1) of split s (of S) of a tile that sees n_kt KV tiles.
+PA_HD void split_range(int64_t n_kt, int s, int S, int64_t* kt0, int64_t* kt1) {
+  *kt0 = (int64_t)s * n_kt / S;
+  *kt1 = (int64_t)(s + 1) * n_kt / S;
+}
+
+// Unit u -> (Q tile, KV head, split). Units run longest first: the last Q tile (most keys)
+// gets the lowest unit indices.
+PA_HD void unit_coords(int64_t u, int64_t q_tiles, int Hkv, int S, int64_t* qt, int* g, int* s) {
+  const int64_t per_tile = (int64_t)Hkv * S;
+  *qt = q_tiles - 1 - u / per_tile;
+  const int64_t rem = u % per_tile;
+  *g = (int)(rem / S);
+  *s = (int)(rem % S);
+}
+
+}  // namespace pa

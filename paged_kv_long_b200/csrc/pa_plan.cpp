@@ -1,0 +1,168 @@
+// pa_plan.cpp — host planner: split count and workspace for one piece.
+//
+// splash PR #33 ("What changed") picks the split count from the GPU's core count, the KV
+// heads and the piece's tiles, so that short pieces at long history still fill the GPU, and
+// sizes the split workspace from it. On B200 one CTA of the prefill kernel owns one SM (it
+// uses ~225 KB of shared memory and the whole 512-column tensor memory), so the question is
+// how the (KV head, Q tile, split) units pack onto 148 SMs. The default policy answers it by
+// simulating the launch: units are dispatched in index order (longest first) to the SM that
+// frees first, and the split count with the smallest simulated makespan plus combine cost
+// wins. The pages' own rule and the earlier rule it replaced are kept as policies.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <functional>
+#include <queue>
+#include <vector>
+
+#include "pa.h"
+#include "pa_geometry.h"
+
+namespace {
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Cost model (microseconds), B200: a 128x128 KV tile costs 4*128*128*D FLOPs at about
+// 1.4 PFLOP/s shared by 148 SMs; a unit pays a fixed start/finish cost (tensor memory
+// allocation, Q tile load, pipeline fill, writing 128 rows of fp32 output); the combine
+// streams S partials through HBM.
+struct CostModel {
+  double tile_us, unit_us, combine_us_per_byte, combine_fixed_us;
+  explicit CostModel(int D) {
+    const double per_sm_flops = 1.4e15 / 148.0;
+    tile_us = 4.0 * pa::kTileKeys * pa::kTileRows * D / per_sm_flops * 1e6;
+    unit_us = 2.0 + pa::kTileRows * (double)D * 4.0 / 60e9 * 1e6;
+    combine_us_per_byte = 1.0 / 5.0e12 * 1e6;
+    combine_fixed_us = 4.0;
+  }
+};
+
+double simulate(int num_sms, int64_t q_tiles, int64_t R, int G, int Hkv, int64_t H, int S,
+                int D) {
+  const CostModel cm(D);
+  std::priority_queue<double, std::vector<double>, std::greater<double>> sms;
+  for (int i = 0; i < num_sms; ++i) sms.push(0.0);
+  double makespan = 0.0;
+  // Units in launch order: last Q tile first; within a tile, KV heads then splits.
+  for (int64_t qt = q_tiles - 1; qt >= 0; --qt) {
+    const int64_t n_kt = pa::tile_kv_tiles(qt, R, G, H);
+    for (int g = 0; g < Hkv; ++g) {
+      for (int s = 0; s < S; ++s) {
+        int64_t kt0, kt1;
+        pa::split_range(n_kt, s, S, &kt0, &kt1);
+        const double w = (kt1 - kt0) * cm.tile_us + cm.unit_us;
+        const double t = sms.top() + w;
+        sms.pop();
+        sms.push(t);
+        makespan = std::max(makespan, t);
+      }
+    }
+  }
+  (void)G;
+  return makespan;
+}
+
+double combine_cost(int S, int64_t R, int Hq, int D) {
+  if (S <= 1) return 0.0;
+  const CostModel cm(D);
+  const double bytes = (double)S * R * Hq * (D + 1) * 4.0 + (double)R * Hq * D * 4.0;
+  return bytes * cm.combine_us_per_byte + cm.combine_fixed_us;
+}
+
+}  // namespace
+
+extern "C" int pa_cores_policy_splits(int cores, int kv_heads, int tiles) {
+  if (cores <= 0 || kv_heads <= 0 || tiles <= 0) return 1;
+  const int target = std::min(256, std::max(32, (32 * cores) / kv_heads));
+  return std::min(32, std::max(1, target / tiles));
+}
+
+extern "C" int pa_legacy_policy_splits(int kv_heads, int tiles) {
+  if (kv_heads <= 0 || tiles <= 0) return 1;
+  return std::min(32, std::max(1, 32 / (tiles * kv_heads)));
+}
+
+extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_size,
+                       int chunk_rows, int64_t hist_len, int dtype, float scale,
+                       int splits_override, int policy, int paged, pa_plan_t* plan) {
+  if (!plan) return PA_ERR_INVALID_ARG;
+  memset(plan, 0, sizeof *plan);
+  if (num_sms <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || chunk_rows <= 0 || hist_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (splits_override < 0 || policy < 0 || policy > PA_POLICY_LEGACY) return PA_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || isinf(scale)) return PA_ERR_INVALID_ARG;
+  if (n_q_heads % n_kv_heads) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (paged && (!is_pow2(page_size) || page_size < 16 || page_size > 128))
+    return PA_ERR_UNSUPPORTED;
+  if (splits_override > PA_MAX_SPLITS) return PA_ERR_UNSUPPORTED;
+  // Tensor-map coordinates are 32-bit: keep every key row index (plus a tile) below 2^31.
+  const int64_t total_keys = hist_len + chunk_rows;
+  if (total_keys + pa::kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+
+  const int G = n_q_heads / n_kv_heads;
+  const int64_t q_tiles = pa::q_tiles_for(chunk_rows, G);
+  if (q_tiles * n_kv_heads * PA_MAX_SPLITS >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  const int64_t max_kt = pa::tile_kv_tiles(q_tiles - 1, chunk_rows, G, hist_len);
+
+  int S = 1;
+  int used_policy = policy;
+  if (splits_override > 0) {
+    S = splits_override;
+    used_policy = -1;
+  } else if (policy == PA_POLICY_CORES) {
+    S = pa_cores_policy_splits(num_sms, n_kv_heads, (int)std::min<int64_t>(q_tiles, 1 << 30));
+  } else if (policy == PA_POLICY_LEGACY) {
+    S = pa_legacy_policy_splits(n_kv_heads, (int)std::min<int64_t>(q_tiles, 1 << 30));
+  } else {
+    double best = 0.0;
+    const int64_t base_units = q_tiles * n_kv_heads;
+    for (int cand = 1; cand <= PA_MAX_SPLITS; ++cand) {
+      if (cand > 1 && cand > max_kt) break;                   // more splits than KV tiles
+      if (cand > 1 && base_units * cand > 16LL * num_sms) break;  // far past filling the GPU
+      const double t = simulate(num_sms, q_tiles, chunk_rows, G, n_kv_heads, hist_len, cand,
+                                head_dim) +
+                       combine_cost(cand, chunk_rows, n_q_heads, head_dim);
+      if (cand == 1 || t < best * 0.98) {  // a new split must win by 2% to be worth it
+        best = t;
+        S = cand;
+      }
+    }
+  }
+
+  plan->num_sms = num_sms;
+  plan->n_q_heads = n_q_heads;
+  plan->n_kv_heads = n_kv_heads;
+  plan->head_dim = head_dim;
+  plan->page_size = paged ? page_size : 0;
+  plan->group = G;
+  plan->chunk_rows = chunk_rows;
+  plan->q_tiles = (int32_t)q_tiles;
+  plan->splits = S;
+  plan->paged = paged ? 1 : 0;
+  plan->dtype = dtype;
+  plan->policy = used_policy;
+  plan->hist_len = hist_len;
+  plan->units = q_tiles * n_kv_heads * S;
+  plan->scale = scale > 0.0f ? scale : (float)(1.0 / sqrt((double)head_dim));
+  plan->est_us = (float)(simulate(num_sms, q_tiles, chunk_rows, G, n_kv_heads, hist_len, S,
+                                  head_dim) +
+                         combine_cost(S, chunk_rows, n_q_heads, head_dim));
+  plan->ws_bytes = S > 1 ? (uint64_t)S * chunk_rows * n_q_heads * (head_dim + 1) * 4ull : 0ull;
+  return PA_OK;
+}
+
+extern "C" const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_CUDA: return "CUDA call failed";
+    case PA_ERR_TIMEOUT: return "a kernel wait timed out";
+    case PA_ERR_PAGE_INDEX: return "page-table entry out of range";
+    default: return "unknown status";
+  }
+}

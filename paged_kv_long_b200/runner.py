@@ -1,0 +1,69 @@
+"""Run a whole workload (a sequence of pieces over one KV cache) through libpa on one GPU.
+
+One step is what a prefill engine does for the chunk's attention: for every piece, plan it
+(host), then pa_prefill and, when the piece is split, pa_combine on the same stream. Plans,
+outputs and the workspace are made once; ``run()`` only enqueues kernels.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import binding
+from .inputs import Inputs
+
+
+def _dev_tensor(bits: np.ndarray, dtype: str, device):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    t = t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+    return t.to(device)
+
+
+class DeviceWorkload:
+    def __init__(self, inp: Inputs, device="cuda", paged: bool = True, splits: int | None = None,
+                 policy: str = "makespan", num_sms: int | None = None):
+        import torch
+        wl = inp.wl
+        self.wl, self.paged, self.device = wl, paged, torch.device(device)
+        self.q = _dev_tensor(inp.q, wl.dtype, self.device)
+        if paged:
+            self.k = _dev_tensor(inp.k_pool, wl.dtype, self.device)
+            self.v = _dev_tensor(inp.v_pool, wl.dtype, self.device)
+            self.table = torch.from_numpy(inp.page_table).to(self.device)
+        else:
+            self.k = _dev_tensor(inp.k_logical, wl.dtype, self.device)
+            self.v = _dev_tensor(inp.v_logical, wl.dtype, self.device)
+            self.table = None
+        if splits is None:
+            splits = wl.splits
+        self.plans = []
+        for h, r in wl.pieces:
+            self.plans.append(binding.plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size,
+                                           r, h, wl.dtype, wl.scale, splits, policy, paged,
+                                           num_sms))
+        self.outs = [torch.empty((r, wl.n_q_heads, wl.head_dim), dtype=torch.float32,
+                                 device=self.device) for _, r in wl.pieces]
+        ws_elems = max(p.ws_bytes for p in self.plans) // 4
+        self.ws = torch.empty(max(ws_elems, 4), dtype=torch.float32, device=self.device)
+
+    def piece_inputs(self, i: int):
+        h, r = self.wl.pieces[i]
+        off = h - self.wl.first_pos
+        q = self.q[off:off + r]
+        if self.paged:
+            return q, self.k, self.v, self.table
+        # contiguous K/V of exactly H+R rows for this piece
+        return q, self.k[:h + r], self.v[:h + r], None
+
+    def run_piece(self, i: int, stream=None):
+        q, k, v, tab = self.piece_inputs(i)
+        p = self.plans[i]
+        binding.prefill(p, q, k, v, tab, self.outs[i], self.ws, stream)
+        binding.combine(p, self.ws, self.outs[i], stream)
+
+    def run(self, stream=None):
+        for i in range(len(self.wl.pieces)):
+            self.run_piece(i, stream)
+
+    def outputs_host(self) -> list[np.ndarray]:
+        return [o.cpu().numpy() for o in self.outs]
