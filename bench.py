@@ -106,43 +106,47 @@ def dist_env():
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
-def oracle_sample_rate(wl, inp, seconds: float, seed: int = 17):
-    """Time the fp64 oracle on a stride sample of (row, head) pairs spread over the whole
-    workload; return (query tok/s estimate, samples, elapsed, threads)."""
-    import numpy as np
-    from oracle import oracle
-    Hq = wl.n_q_heads
-    pieces = wl.pieces
-    total_rows = sum(r for _, r in pieces)
+class OracleSampler:
+    """The fp64 CPU oracle timed on a stride sample of (row, head) pairs spread over the whole
+    workload (one random head per sampled row), scaled to query tokens/s."""
 
-    def run(n):
+    def __init__(self, wl, inp):
+        from oracle import oracle
+        self.oracle, self.wl, self.inp = oracle, wl, inp
+        self.threads = oracle.max_threads()
+
+    def run(self, n: int, seed: int = 17):
+        import numpy as np
+        wl, inp, oracle = self.wl, self.inp, self.oracle
+        pieces = wl.pieces
         rng = np.random.default_rng(seed)
         t_sum, pairs = 0.0, 0
-        # stride sample across the workload's query rows, one random head each
+        total_rows = sum(r for _, r in pieces)
         gidx = np.linspace(0, total_rows - 1, n).astype(np.int64)
         starts = np.cumsum([0] + [r for _, r in pieces])
         for i, (h, r) in enumerate(pieces):
             sel = gidx[(gidx >= starts[i]) & (gidx < starts[i + 1])] - starts[i]
             if len(sel) == 0:
                 continue
-            heads = rng.integers(0, Hq, size=len(sel)).astype(np.int32)
-            q = inp.piece_q(i)
-            pb = oracle.Problem(q=q, k=inp.k_pool, v=inp.v_pool, hist_len=h, dtype=wl.dtype,
-                                page_table=inp.page_table, scale=wl.scale)
+            heads = rng.integers(0, wl.n_q_heads, size=len(sel)).astype(np.int32)
+            pb = oracle.Problem(q=inp.piece_q(i), k=inp.k_pool, v=inp.v_pool, hist_len=h,
+                                dtype=wl.dtype, page_table=inp.page_table, scale=wl.scale)
             t0 = time.perf_counter()
             oracle.attend(pb, sel, heads)
             t_sum += time.perf_counter() - t0
             pairs += len(sel)
-        return t_sum, pairs
+        # one (row, head) pair is 1/Hq of a query token's attention
+        return (pairs / wl.n_q_heads) / t_sum, pairs, t_sum
 
-    threads = oracle.max_threads()
-    t_cal, p_cal = run(max(8, threads))
-    per_pair = t_cal / max(p_cal, 1)
-    n = int(max(p_cal, min(200000, seconds / max(per_pair, 1e-9))))
-    t, pairs = run(n)
-    # one (row, head) pair is 1/Hq of a query token's attention
-    tok_s = (pairs / Hq) / t
-    return tok_s, pairs, t, threads
+    def calibrate(self, seconds: float) -> int:
+        """Sample size that costs about `seconds` of CPU time."""
+        n = max(8, self.threads)
+        while True:
+            _, pairs, t = self.run(n)
+            if t >= seconds / 4 or n >= 200000:
+                break
+            n *= 2
+        return int(max(8, min(200000, n * seconds / max(t, 1e-6))))
 
 
 def reference_arm(args):
@@ -153,14 +157,16 @@ def reference_arm(args):
     wl = WORKLOADS[args.workload]
     inp = generate(wl, poison=False)
     steps, warmup = args.steps, args.warmup
-    per_step = max(2.0, min(10.0, 150.0 / max(steps + warmup, 1)))
-    for _ in range(warmup):
-        oracle_sample_rate(wl, inp, per_step / 4)
-    rates, times, cores, pairs = [], [], 1, 0
+    per_step = max(1.0, min(10.0, 80.0 / max(steps + warmup, 1)))
+    sampler = OracleSampler(wl, inp)
+    n = sampler.calibrate(per_step)
+    for k in range(warmup):
+        sampler.run(max(8, n // 4), seed=50 + k)
+    rates, pairs = [], 0
     for k in range(steps):
-        r, pairs, t, cores = oracle_sample_rate(wl, inp, per_step, seed=100 + k)
+        r, pairs, _ = sampler.run(n, seed=100 + k)
         rates.append(r)
-        times.append(t)
+    cores = sampler.threads
     value = statistics.median(rates)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -275,8 +281,9 @@ def gpu_arm(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     split_arg = args.splits if args.splits is not None else None
-    dw = DeviceWorkload(inp, dev, paged=True, splits=split_arg, policy=args.policy)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    paged = args.layout == "paged"
+    dw = DeviceWorkload(inp, dev, paged=paged, splits=split_arg, policy=args.policy)
+    flush = torch.empty(max(args.l2_flush_mb, 1) * (1 << 20) // 4, dtype=torch.float32, device=dev)
     peaks = load_peaks()
 
     def barrier():
@@ -309,22 +316,24 @@ def gpu_arm(args):
     t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
 
     # ---- contiguous control at the same split counts (the ratio's denominator)
-    dwc = DeviceWorkload(inp, dev, paged=False, splits=None, policy=args.policy)
-    for i, p in enumerate(dw.plans):   # same S per piece as the paged run
+    t_contig = last_paged = last_contig = None
+    if paged and not args.no_contiguous:
         from paged_kv_long_b200 import binding
-        h, r = wl.pieces[i]
-        dwc.plans[i] = binding.plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size, r, h,
-                                    wl.dtype, wl.scale, p.splits, "makespan", False)
-    c_ms, c_kern = time_steps(dwc, max(3, args.steps // 2), args.warmup, flush, stream,
-                              record_kernels=True)
-    t_contig = sum(c_ms) / len(c_ms)
-    last_paged = statistics.median(k[-1] for k in kern_ms)
-    last_contig = statistics.median(k[-1] for k in c_kern)
-    del dwc
+        dwc = DeviceWorkload(inp, dev, paged=False, splits=None, policy=args.policy)
+        for i, p in enumerate(dw.plans):   # same S per piece as the paged run
+            h, r = wl.pieces[i]
+            dwc.plans[i] = binding.plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size, r,
+                                        h, wl.dtype, wl.scale, p.splits, "makespan", False)
+        c_ms, c_kern = time_steps(dwc, max(3, args.steps // 2), args.warmup, flush, stream,
+                                  record_kernels=True)
+        t_contig = sum(c_ms) / len(c_ms)
+        last_paged = statistics.median(k[-1] for k in kern_ms)
+        last_contig = statistics.median(k[-1] for k in c_kern)
+        del dwc
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and paged:
         e_ms, h2d, d2h = e2e_steps(inp, dw, max(2, min(args.steps, 5)), stream)
         t_e = sum(e_ms) / len(e_ms)
         e2e = {"value": world * tokens / (t_e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -334,8 +343,9 @@ def gpu_arm(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r, pairs, t, cores = oracle_sample_rate(wl, inp, args.cpu_seconds)
-        cpu = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
+        sampler = OracleSampler(wl, inp)
+        r, pairs, t = sampler.run(sampler.calibrate(args.cpu_seconds))
+        cpu = {"value": r, "unit": UNIT, "cores": sampler.threads, "kind": "oracle",
                "sample": f"{pairs} (row, head) pairs stride-sampled over all {wl.query_rows} query "
                          f"rows of the workload, {t:.1f} s of fp64 CPU work, scaled to tok/s"}
 
@@ -351,13 +361,13 @@ def gpu_arm(args):
         "config": {"workload": wl.name, "seq_len": wl.total_keys, "chunk_rows": wl.pieces[0][1],
                    "pieces": len(wl.pieces), "n_q_heads": wl.n_q_heads,
                    "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
-                   "page_size": wl.page_size, "kv_layout": "paged",
+                   "page_size": wl.page_size, "kv_layout": args.layout,
                    "splits": [p.splits for p in dw.plans], "split_policy": args.policy,
-                   "l2": "flushed between steps (512 MiB write outside the timed events)",
+                   "l2": f"flushed between steps ({args.l2_flush_mb} MiB write outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "tflops": tflops,
-        "paged_contiguous_ratio": t_contig / t_step,
-        "paged_contiguous_ratio_last_chunk": last_contig / last_paged,
+        "paged_contiguous_ratio": (t_contig / t_step) if t_contig else None,
+        "paged_contiguous_ratio_last_chunk": (last_contig / last_paged) if t_contig else None,
         "contiguous_ms_per_step": t_contig,
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": None,
@@ -378,13 +388,16 @@ def gpu_arm(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c5", choices=["c1", "c2", "c3", "c4", "c5"])
     ap.add_argument("--splits", type=int, default=None,
                     help="split count for every piece (default: the workload's, else the planner)")
     ap.add_argument("--policy", default="makespan", choices=["makespan", "cores", "legacy"])
+    ap.add_argument("--layout", default="paged", choices=["paged", "contiguous"])
+    ap.add_argument("--no-contiguous", action="store_true", help="skip the contiguous control")
+    ap.add_argument("--l2-flush-mb", type=int, default=L2_FLUSH_BYTES >> 20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
