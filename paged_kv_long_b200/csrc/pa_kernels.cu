@@ -4,14 +4,16 @@
 //   The operation is prefill attention of a query chunk against a long history read through
 //   a paged KV cache (BaseRT issue #51, "Results"), with the history of a piece cut into
 //   splits whose partials a reduce merges (splash PR #33, "What changed"). The B200 design:
-//   * warp 4 (producer) reads the page table and issues one TMA box per (page, 64-wide
-//     D panel) into a ring of 16 KB, 128-byte-swizzled shared-memory panels;
-//   * warp 5 (MMA) issues tcgen05.mma: S = Q K^T into one of two tensor-memory S buffers,
-//     then O += P V into a tensor-memory O accumulator (fp32);
+//   * warp 4 (producer) reads the page table and issues TMA boxes into a ring of 16 KB,
+//     128-byte-swizzled shared-memory panels: K as one box per (page, 64-wide D panel), V as
+//     one box per (page, half of D);
+//   * warp 5 (MMA) issues tcgen05.mma: S = Q K^T into one of two tensor-memory S buffers
+//     (Q and K from shared memory), then O += P V with P read from tensor memory where the
+//     softmax wrote it over its own S buffer (fp32 accumulation in tensor memory);
 //   * warps 0-3 (softmax, one thread per packed Q row = tensor-memory lane) load the GQA-
 //     packed Q tile, read S with tcgen05.ld, apply the causal mask by select, keep the
 //     running max and sum (rescaling O only when the max grows by more than 2^8), write P
-//     (rounded to the input type) to shared memory, and finally write O / l (fp32) or the
+//     (rounded to the input type) to tensor memory, and finally write O / l (fp32) or the
 //     split partial and its base-2 log-sum-exp.
 //   Every wait is bounded: on expiry the kernel sets the timeout bit, abandons its work,
 //   waits for its own copies and MMAs in flight, frees tensor memory and exits.
@@ -24,6 +26,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -37,12 +40,15 @@ __device__ unsigned int g_pa_error_flags;
 constexpr unsigned kFlagPage = 1u;
 constexpr unsigned kFlagTimeout = 2u;
 
-constexpr int kPanel = 128 * 128;          // bytes of one 128-row x 128-byte panel
-constexpr int kThreads = 192;              // 4 softmax warps, 1 producer warp, 1 MMA warp
+constexpr int kPanel = 128 * 128;          // bytes of one 128-row x 128-byte panel (a slot)
+constexpr int kThreads = 256;  // 4 softmax warps, 1 MMA warp, 3 TMA-issuing warps
+constexpr int kIssuers = 3;    // TMA issue latency is per issuing warp: three overlap it
+constexpr int kMmaWarp = 4;
 constexpr float kRescaleLog2 = 8.0f;       // rescale O only when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 0;              // O accumulator: columns [0, D)
 constexpr uint32_t kSCol0 = 256;           // S buffers: [256, 384) and [384, 512)
+constexpr uint32_t kPColOff = 64;          // P (16-bit pairs) over the upper half of its S
 
 struct PrefillArgs {
   const uint16_t* q;
@@ -55,37 +61,71 @@ struct PrefillArgs {
   int64_t total_keys;
   int32_t R, Hq, Hkv, G;
   int32_t q_tiles, splits;
-  int32_t page_size;
+  int32_t page_rows;     // key rows per page: the page size, or kTileKeys when contiguous
+  int32_t page_shift;    // log2(page_rows)
   int32_t pages_per_tile;
+  int32_t v_rows;        // key rows per V box (<= page_rows; a box is at most one slot)
+  int32_t v_shift;       // log2(v_rows)
   int32_t num_pages;
   int32_t oob_row;       // a key-row coordinate past the pool: the TMA fills zeros there
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
 };
 
+// Shared-memory layout. The ring holds 16 KB slots, filled and consumed in the order K0, K1,
+// V0, K2, V1, ..., V_{n-1}; every K or V tile takes NP consecutive slots (mod NSLOT). A K
+// tile is one 64-wide D panel per slot (128 keys x 128 B, the K-major B operand of Q K^T),
+// loaded as one TMA box per (page, panel). A V tile is a run of TMA boxes of v_rows keys x
+// all NP panels (each box panel-major, the MN-major B operand of P V); a box never straddles
+// two slots. Fill number q is issued by TMA warp q % kIssuers.
 template <int D>
 struct Cfg {
-  static constexpr int NP = D / 64;                 // 64-element panels per K/V/Q row
-  static constexpr int NSLOT = (D == 256) ? 8 : 10; // ring of 16 KB panels (multiple of NP)
+  static constexpr int NP = D / 64;                  // 64-element panels per K/V/Q row
+  static constexpr int NSLOT = (D == 256) ? 10 : 12; // ring of 16 KB slots
   static constexpr int Q_OFF = 0;
-  static constexpr int P_OFF = Q_OFF + NP * kPanel;
-  static constexpr int RING_OFF = P_OFF + 2 * kPanel;
+  static constexpr int RING_OFF = Q_OFF + NP * kPanel;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * kPanel;
-  // barriers: full[NSLOT], empty[NSLOT], q_full, s_full[2], s_free[2], p_full, pv_done, mma_done
+  // barriers: full[NSLOT], empty[NSLOT], q_full, s_full[2], p_full[2], pv_done, mma_done
   static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_QFULL = 2 * NSLOT, B_SFULL = 2 * NSLOT + 1,
-                       B_SFREE = 2 * NSLOT + 3, B_PFULL = 2 * NSLOT + 5,
-                       B_PVDONE = 2 * NSLOT + 6, B_MMADONE = 2 * NSLOT + 7, N_BARS = 2 * NSLOT + 8;
+                       B_PFULL = 2 * NSLOT + 3, B_PVDONE = 2 * NSLOT + 5,
+                       B_MMADONE = 2 * NSLOT + 6, N_BARS = 2 * NSLOT + 7;
   static constexpr int MISC_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int SMEM = MISC_OFF + 16;
-  static constexpr int LAUNCH_SMEM = SMEM + 1024;   // slack to align the base to 1024 B
-  static_assert(NSLOT % NP == 0, "a V tile's panels must not wrap around the ring");
+  static constexpr int LAUNCH_SMEM = SMEM + 1024;    // slack to align the base to 1024 B
+  static constexpr int PANEL_LOG = (NP == 4) ? 9 : (NP == 2) ? 8 : 7;  // log2(NP * 128)
   static_assert(LAUNCH_SMEM <= 232448, "exceeds 227 KB of shared memory per CTA");
 };
 
-// Position of tile j's V panels in the load order K0, K1, V0, K2, V1, ..., V_{n-1}.
+// Position of tile j's V in the load order K0, K1, V0, K2, V1, ..., V_{n-1}.
 __device__ __forceinline__ uint32_t v_item(int j, int n) {
   return j == n - 1 ? 2u * n - 1u : 2u * j + 2u;
 }
+
+// Byte offset, inside a V tile, of (key row k of the tile, panel p).
+template <int NP, int PANEL_LOG>
+__device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift) {
+  return ((k >> v_shift) << (v_shift + PANEL_LOG)) + ((p << v_shift) << 7) +
+         ((k & ((1u << v_shift) - 1u)) << 7);
+}
+
+#ifdef PA_TRACE
+// Instrumented builds only: cycle counters summed over all CTAs (see pa_trace_read), and an
+// event log of the first CTAs: (kind << 56 | cta << 48 | index << 32 | clock low 32 bits).
+__device__ unsigned long long g_pa_trace[16];
+constexpr int kLogCap = 1 << 16;  // 2 CTAs x 3 roles x 8192 events
+__device__ unsigned long long g_pa_log[kLogCap];
+// role: 0 producer, 1 MMA, 2 softmax; `n` is the role's own event counter (no atomics).
+__device__ __forceinline__ void tlog(int role, unsigned& n, int kind, int index) {
+  const unsigned long long clk = (unsigned)clock64();
+  if (blockIdx.x < 2 && n < 8192u)
+    g_pa_log[(blockIdx.x * 3 + role) * 8192 + n++] =
+        ((unsigned long long)kind << 56) | ((unsigned long long)blockIdx.x << 48) |
+        ((unsigned long long)(index & 0xFFFF) << 32) | clk;
+}
+#define PA_TRACE_ONLY(...) __VA_ARGS__
+#else
+#define PA_TRACE_ONLY(...)
+#endif
 
 // ---------------------------------------------------------------- bounded waits
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -104,6 +144,12 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile i
   }
 }
 
+// One thread waits (the single-lane roles).
+__device__ __forceinline__ bool thread_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            uint64_t timeout_ns) {
+  return mbar_try_wait(bar, parity) || wait_slow(bar, parity, abort_flag, timeout_ns, true);
+}
+
 // All 32 lanes wait; the result is uniform across the warp.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t timeout_ns) {
@@ -115,18 +161,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            uint64_t timeout_ns) {
   if (!mbar_try_wait(bar, parity)) wait_slow(bar, parity, abort_flag, timeout_ns, false);
-  __syncwarp();
 }
 
 template <bool BF16>
-__device__ __forceinline__ uint32_t pack_round(float a, float b, float& sum) {
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
   if constexpr (BF16) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    sum += __low2float(h) + __high2float(h);
     return *reinterpret_cast<const uint32_t*>(&h);
   } else {
     const __half2 h = __floats2half2_rn(a, b);
-    sum += __low2float(h) + __high2float(h);
     return *reinterpret_cast<const uint32_t*>(&h);
   }
 }
@@ -168,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   auto bar = [&](int i) -> uint32_t { return sb + C::BAR_OFF + 8u * (uint32_t)i; };
+  auto slot_addr = [&](uint32_t slot) -> uint32_t { return sb + C::RING_OFF + slot * kPanel; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 4);
 
@@ -179,20 +223,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(C::B_QFULL), 4);
     mbar_init(bar(C::B_SFULL + 0), 1);
     mbar_init(bar(C::B_SFULL + 1), 1);
-    mbar_init(bar(C::B_SFREE + 0), 4);
-    mbar_init(bar(C::B_SFREE + 1), 4);
-    mbar_init(bar(C::B_PFULL), 4);
+    mbar_init(bar(C::B_PFULL + 0), 4);
+    mbar_init(bar(C::B_PFULL + 1), 4);
     mbar_init(bar(C::B_PVDONE), 1);
     mbar_init(bar(C::B_MMADONE), 1);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kMmaWarp + 1 && lane == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -201,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
+  PA_TRACE_ONLY(long long tr[4] = {0, 0, 0, 0}; const long long t_begin = clock64(); unsigned tln = 0;)
 
   if (warp < 4) {
     // ============================================================ softmax + epilogue
@@ -229,26 +273,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int64_t limit = valid ? a.hist_len + tok : -1;  // last key this row may see
     const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     float m_run = -INFINITY;  // running max of scale*log2(e)*score
-    float l_run = 0.f;        // running sum of the rounded probabilities
+    float l_run = 0.f;        // running sum of the probabilities (fp32)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int sbuf = j & 1;
+      const uint32_t s_col = kSCol0 + 128u * sbuf;
       const int64_t key0 = (kt0 + j) * kTileKeys;
+      PA_TRACE_ONLY(long long tw = clock64();)
       if (!warp_wait(bar(C::B_SFULL + sbuf), (j >> 1) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
+      PA_TRACE_ONLY(const long long tc = clock64(); tr[0] += tc - tw;
+                    if (threadIdx.x == 0) tlog(2, tln, 8, j);)
       tc_fence_after();
       float sv[kTileKeys];
 #pragma unroll
       for (int c = 0; c < kTileKeys / 32; ++c)
-        tmem_ld32(t_lane + kSCol0 + 128u * sbuf + 32u * c,
-                  *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
+        tmem_ld32(t_lane + s_col + 32u * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_SFREE + sbuf));
 
       // causal mask by select (masked scores become -inf, whatever bits they held)
       const int64_t rel64 = limit - key0;
@@ -258,11 +303,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kTileKeys; ++c)
           if (c > rel) sv[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max: eight independent chains, then a tree
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < kTileKeys; ++c) mx = fmaxf(mx, sv[c]);
+      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+#pragma unroll
+      for (int c = 8; c < kTileKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m_run, mx * a.scale_log2);
       const bool need = m_new > m_run + kRescaleLog2;
+      // pv_done completes once per PV MMA group, in order. Parity waits are only sound when
+      // no phase is skipped, so every tile j >= 1 observes PV_{j-1} before it releases P_j
+      // (PV_j cannot finish before that); here early when O must be rescaled, else below.
+      bool pv_prev_seen = (j == 0);
       if (j == 0) {
         if (need) m_run = m_new;
       } else if (__any_sync(0xffffffffu, need)) {
@@ -271,9 +325,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+        pv_prev_seen = true;
         tc_fence_after();
         const float f = need ? ex2(m_run - m_new) : 1.0f;
         l_run *= f;
+        PA_TRACE_ONLY(tr[3] += 1;)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
@@ -287,21 +343,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (need) m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      uint32_t pk[kTileKeys / 2];
-      float lsum = 0.f;
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kTileKeys; c += 2) {
-        const float p0 = ex2(fmaf(sv[c], a.scale_log2, -m_use));
-        const float p1 = ex2(fmaf(sv[c + 1], a.scale_log2, -m_use));
-        pk[c / 2] = pack_round<BF16>(p0, p1, lsum);
+      for (int h = 0; h < 2; ++h) {  // two 64-key halves -> 32 columns of P each
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 x = ffma2(make_float2(sv[64 * h + c], sv[64 * h + c + 1]), sc2, nm2);
+          const float2 pr = make_float2(ex2(x.x), ex2(x.y));
+          ls[(c >> 1) & 3] = fadd2(ls[(c >> 1) & 3], pr);
+          pk[c >> 1] = pack2<BF16>(pr.x, pr.y);
+        }
+        tmem_st32u(t_lane + s_col + kPColOff + 32u * h, pk);
       }
-      l_run += lsum;
-
-      // P is single-buffered: PV of the previous tile must be done reading it.
-      if (j >= 1 && !warp_wait(bar(C::B_PVDONE), (j - 1) & 1, abort_flag, tmo)) {
+      l_run += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y) + (ls[2].x + ls[2].y) +
+               (ls[3].x + ls[3].y);
+      if (!pv_prev_seen && !warp_wait(bar(C::B_PVDONE), (j - 1) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
+
       if constexpr (PAGED) {
         // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but
         // 0 * NaN is NaN inside the MMA, so those V rows are zeroed before PV reads them.
@@ -317,27 +380,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (key0 + r >= a.total_keys) {
             for (int p = 0; p < NP; ++p) {
-              const uint32_t row_addr =
-                  sb + C::RING_OFF + ((seq0 + p) % NSLOT) * kPanel + r * 128;
+              const uint32_t off = v_offset<NP, C::PANEL_LOG>((uint32_t)r, p, a.v_shift);
+              const uint32_t ra = slot_addr((seq0 + (off >> 14)) % NSLOT) + (off & (kPanel - 1));
 #pragma unroll
-              for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + c * 16, 0u, 0u, 0u, 0u);
+              for (int c = 0; c < 8; ++c) st_shared_v4(ra + c * 16, 0u, 0u, 0u, 0u);
             }
+            fence_proxy_async_smem();
           }
         }
       }
-      // P row -> shared memory: two 64-key K-major panels, 128-byte swizzle.
-#pragma unroll
-      for (int c = 0; c < kTileKeys / 8; ++c) {
-        const int pp = c >> 3, cc = c & 7;
-        st_shared_v4(sb + C::P_OFF + pp * kPanel + r * 128 + ((cc ^ (r & 7)) << 4), pk[4 * c],
-                     pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_PFULL));
+      if (lane == 0) mbar_arrive(bar(C::B_PFULL + sbuf));
+      PA_TRACE_ONLY(tr[1] += clock64() - tc; if (threadIdx.x == 0) tlog(2, tln, 9, j);)
     }
 
+    PA_TRACE_ONLY(const long long te = clock64();)
     if (ok) ok = warp_wait(bar(C::B_PVDONE), (n - 1) & 1, abort_flag, tmo);
     if (ok) {
       tc_fence_after();
@@ -361,133 +420,193 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.ws_lse[((int64_t)s * a.R + tok) * a.Hq + head] =
             l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
     }
-  } else if (warp == 4) {
-    // ============================================================ TMA producer
-    const int ppt = PAGED ? a.pages_per_tile : 1;
-    uint32_t seq = 0;
+    PA_TRACE_ONLY(tr[2] += clock64() - te;
+                  if (lane == 0) {
+                    atomicAdd(&g_pa_trace[6], (unsigned long long)tr[0]);
+                    atomicAdd(&g_pa_trace[7], (unsigned long long)tr[1]);
+                    atomicAdd(&g_pa_trace[8], (unsigned long long)tr[2]);
+                    atomicAdd(&g_pa_trace[9], (unsigned long long)tr[3]);
+                    atomicAdd(&g_pa_trace[10], (unsigned long long)(clock64() - t_begin));
+                    if (warp == 0) atomicAdd(&g_pa_trace[11], (unsigned long long)n);
+                  })
+  } else if (warp > kMmaWarp) {
+    // ============================================================ TMA issuers (three warps)
+    const int w = warp - kMmaWarp - 1;  // this warp issues fill numbers q with q % kIssuers == w
+    const int ppt = a.pages_per_tile;   // pages per KV tile (1 when contiguous)
+    const int prow = a.page_rows;       // key rows per page (kTileKeys when contiguous)
+    const int vsub = prow >> a.v_shift; // V boxes per page
+    const int vbytes_log = a.v_shift + C::PANEL_LOG;   // log2 of a V box's bytes
+    const int vbox_per_slot = 1 << (14 - vbytes_log);
     bool ok = true;
-    // Raw page-table entries of this lane's page in tiles j-1, j, j+1 (read one tile ahead).
+    // Lane i < ppt holds the key-row coordinate of page i of a tile (read one tile ahead).
     auto fetch = [&](int jt) -> int32_t {
-      if (!PAGED || jt >= n || lane >= ppt) return -1;
-      const int64_t lp = (kt0 + jt) * ppt + lane;
-      return lp < a.table_len ? __ldg(a.page_table + lp) : -1;
-    };
-    auto load_item = [&](const CUtensorMap* map, int jt, int32_t entry) -> bool {
-      int32_t row_lane = a.oob_row;
+      int32_t row = a.oob_row;
       if constexpr (PAGED) {
         const int64_t lp = (kt0 + jt) * ppt + lane;
-        if (lane < ppt && lp < a.table_len) {
-          if (entry >= 0 && entry < a.num_pages)
-            row_lane = entry * a.page_size;
-          else
+        if (jt < n && lane < ppt && lp < a.table_len) {
+          const int32_t e = __ldg(a.page_table + lp);
+          if (e >= 0 && e < a.num_pages)
+            row = e << a.page_shift;
+          else if (w == 0)
             atomicOr(&g_pa_error_flags, kFlagPage);
         }
+      } else {
+        row = (int32_t)((kt0 + jt) * kTileKeys);
       }
-      const int32_t key0 = (int32_t)((kt0 + jt) * kTileKeys);
-      for (int p = 0; p < NP; ++p) {
-        const uint32_t slot = seq % NSLOT;
-        if (seq >= (uint32_t)NSLOT &&
-            !warp_wait(bar(C::B_EMPTY + slot), ((seq / NSLOT) - 1) & 1, abort_flag, tmo))
-          return false;
-        int32_t rows[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) rows[i] = __shfl_sync(0xffffffffu, row_lane, i);
-        if (lane == 0) {
-          const uint32_t full = bar(C::B_FULL + slot);
-          const uint32_t dst = sb + C::RING_OFF + slot * kPanel;
-          mbar_arrive_expect_tx(full, kPanel);
-          if constexpr (PAGED) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              if (i < ppt) tma_load_3d(dst + i * a.page_size * 128, map, full, p * 64, g, rows[i]);
-          } else {
-            tma_load_3d(dst, map, full, p * 64, g, key0);
-          }
-        }
-        __syncwarp();
-        ++seq;
-      }
-      return true;
+      return row;
     };
-    int32_t e_prev = -1, e_cur = fetch(0), e_next = fetch(1);
+    // Wait until fill q's slot is free and announce its bytes; false if the wait gave up.
+    auto acquire = [&](uint32_t q) -> bool {
+      const uint32_t slot = q % NSLOT;
+      PA_TRACE_ONLY(const long long tw = clock64();)
+      bool r_ok = q < (uint32_t)NSLOT ||
+                  warp_wait(bar(C::B_EMPTY + slot), ((q / NSLOT) - 1) & 1, abort_flag, tmo);
+      PA_TRACE_ONLY(tr[0] += clock64() - tw;)
+      if (r_ok && lane == 0) mbar_arrive_expect_tx(bar(C::B_FULL + slot), kPanel);
+      __syncwarp();
+      return r_ok;
+    };
+    int32_t row_prev = a.oob_row, row_cur = fetch(0), row_next = fetch(1);
+    uint32_t issued_end = 0;  // one past the last fill number this warp issued
     for (int j = 0; j <= n && ok; ++j) {
-      if (j < n) ok = load_item(&tm_k, j, e_cur);
-      if (ok && j >= 1) ok = load_item(&tm_v, j - 1, e_prev);
-      e_prev = e_cur;
-      e_cur = e_next;
-      e_next = fetch(j + 2);
-    }
-    // Every issued copy must land before the CTA may exit.
-    for (uint32_t qn = seq > (uint32_t)NSLOT ? seq - NSLOT : 0; qn < seq; ++qn)
-      drain_wait(bar(C::B_FULL + qn % NSLOT), (qn / NSLOT) & 1, abort_flag, tmo);
-  } else {
-    // ============================================================ MMA issuer
-    const uint32_t idesc_qk = umma_idesc_f16(128, kTileKeys, BF16, false);
-    const uint32_t idesc_pv = umma_idesc_f16(128, D, BF16, true);
-    bool ok = warp_wait(bar(C::B_QFULL), 0, abort_flag, tmo);
-    tc_fence_after();
-    uint32_t seq = 0;
-    for (int j = 0; j <= n && ok; ++j) {
-      if (j < n) {
-        const int sbuf = j & 1;
-        if (j >= 2) {
-          ok = warp_wait(bar(C::B_SFREE + sbuf), ((j - 2) >> 1) & 1, abort_flag, tmo);
-          if (!ok) break;
-          tc_fence_after();
+      if (j < n) {  // K tile j: panel k in fill q, one box per page (lane i: page i)
+        const uint32_t item = j == 0 ? 0u : 2u * j - 1u;
+        for (int k = 0; k < NP && ok; ++k) {
+          const uint32_t q = item * NP + k;
+          if ((int)(q % kIssuers) != w) continue;
+          if (!(ok = acquire(q))) break;
+          const uint32_t slot = q % NSLOT;
+          if (lane < ppt)
+            tma_load_3d(slot_addr(slot) + lane * prow * 128, &tm_k, bar(C::B_FULL + slot), k * 64,
+                        g, row_cur);
+          issued_end = q + 1;
+          PA_TRACE_ONLY(if (lane == 0) tlog(0, tln, 1, q);)
         }
-        for (int p = 0; p < NP; ++p) {
-          const uint32_t slot = seq % NSLOT;
-          ok = warp_wait(bar(C::B_FULL + slot), (seq / NSLOT) & 1, abort_flag, tmo);
-          if (!ok) break;
-          tc_fence_after();
-          if (lane == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_ss(tmem + kSCol0 + 128u * sbuf,
-                      smem_desc_sw128(sb + C::Q_OFF + p * kPanel + kk * 32, 16, 1024),
-                      smem_desc_sw128(sb + C::RING_OFF + slot * kPanel + kk * 32, 16, 1024),
-                      idesc_qk, (p | kk) != 0);
-            umma_commit(bar(C::B_EMPTY + slot));
-          }
-          __syncwarp();
-          ++seq;
-        }
-        if (!ok) break;
-        if (lane == 0) umma_commit(bar(C::B_SFULL + sbuf));
-        __syncwarp();
       }
-      if (j >= 1) {
-        const int i = j - 1;
-        ok = warp_wait(bar(C::B_PFULL), i & 1, abort_flag, tmo);
-        for (int p = 0; p < NP && ok; ++p)
-          ok = warp_wait(bar(C::B_FULL + (seq + p) % NSLOT), ((seq + p) / NSLOT) & 1, abort_flag,
-                         tmo);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t slot0 = seq % NSLOT;
-        if (lane == 0) {
-#pragma unroll
-          for (int ks = 0; ks < kTileKeys / 16; ++ks)
-            umma_ss(tmem + kOCol,
-                    smem_desc_sw128(sb + C::P_OFF + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024),
-                    smem_desc_sw128(sb + C::RING_OFF + slot0 * kPanel + ks * 2048, kPanel, 1024),
-                    idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-          for (int p = 0; p < NP; ++p) umma_commit(bar(C::B_EMPTY + (seq + p) % NSLOT));
-          umma_commit(bar(C::B_PVDONE));
+      if (ok && j >= 1) {  // V tile j-1: slot k holds boxes k*vbox_per_slot + lane
+        const uint32_t item = v_item(j - 1, n);
+        for (int k = 0; k < NP && ok; ++k) {
+          const uint32_t q = item * NP + k;
+          if ((int)(q % kIssuers) != w) continue;
+          if (!(ok = acquire(q))) break;
+          const uint32_t slot = q % NSLOT;
+          const int b = k * vbox_per_slot + lane;        // box index inside the V tile
+          const int pg = b / vsub, sub = b - pg * vsub;  // its page and place in the page
+          const int32_t prow_b = __shfl_sync(0xffffffffu, row_prev, pg & 31);
+          if (lane < vbox_per_slot)
+            tma_load_4d(slot_addr(slot) + (lane << vbytes_log), &tm_v, bar(C::B_FULL + slot), 0,
+                        prow_b + (sub << a.v_shift), 0, g);
+          issued_end = q + 1;
+          PA_TRACE_ONLY(if (lane == 0) tlog(0, tln, 2, q);)
         }
-        __syncwarp();
-        seq += NP;
       }
+      row_prev = row_cur;
+      row_cur = row_next;
+      row_next = fetch(j + 2);
     }
-    // Every issued MMA must finish before tensor memory is freed.
-    if (lane == 0) umma_commit(bar(C::B_MMADONE));
+    // Every copy must land before the CTA may exit. Only the last fill of each slot is still
+    // waitable by parity (an earlier one may be two phases back), so each warp waits for its
+    // own fills among the last NSLOT of the whole sequence; fills it never issued (after an
+    // abort) are skipped.
+    const uint32_t all_fills = 2u * n * NP;
+    for (uint32_t q = all_fills > (uint32_t)NSLOT ? all_fills - NSLOT : 0; q < issued_end; ++q)
+      if ((int)(q % kIssuers) == w)
+        drain_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo);
     __syncwarp();
-    drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
+    PA_TRACE_ONLY(if (lane == 0 && w == 0) {
+      atomicAdd(&g_pa_trace[4], (unsigned long long)tr[0]);
+      atomicAdd(&g_pa_trace[5], (unsigned long long)(clock64() - t_begin));
+    })
+  } else {
+    // ============================================================ MMA issuer (one lane)
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_f16(128, kTileKeys, BF16, false);
+      constexpr uint32_t idesc_pv = umma_idesc_f16(128, D, BF16, true);
+      constexpr uint32_t kSlotDesc = kPanel >> 4;  // descriptor units per slot
+      // Descriptor templates; the start address field takes plain additions of (bytes >> 4).
+      const uint64_t q_desc = smem_desc_sw128(sb + C::Q_OFF, 16, 1024);
+      const uint64_t k_desc = smem_desc_sw128(sb + C::RING_OFF, 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(sb + C::RING_OFF, (uint32_t)a.v_rows * 128u, 1024);
+      uint32_t slot = 0, round = 0;
+      bool ok = thread_wait(bar(C::B_QFULL), 0, abort_flag, tmo);
+      tc_fence_after();
+      for (int j = 0; j <= n && ok; ++j) {
+        if (j < n) {
+          // S_j is written over S_{j-2} and its P: the PV MMA that read that P was issued
+          // earlier by this thread, and tcgen05.mma executes in issue order.
+          const uint32_t s_tmem = tmem + kSCol0 + 128u * (j & 1);
+#pragma unroll
+          for (int p = 0; p < NP; ++p) {
+            PA_TRACE_ONLY(const long long tw = clock64();)
+            ok = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
+            PA_TRACE_ONLY(tr[0] += clock64() - tw; tlog(1, tln, 3, j * 16 + p);)
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t ad = q_desc + p * kSlotDesc, bd = k_desc + slot * kSlotDesc;
+            umma_ss(s_tmem, ad, bd, idesc_qk, p != 0 ? 1u : 0u);
+            umma_ss(s_tmem, ad + 2, bd + 2, idesc_qk, 1u);
+            umma_ss(s_tmem, ad + 4, bd + 4, idesc_qk, 1u);
+            umma_ss(s_tmem, ad + 6, bd + 6, idesc_qk, 1u);
+            umma_commit(bar(C::B_EMPTY + slot));
+            if (++slot == (uint32_t)NSLOT) {
+              slot = 0;
+              ++round;
+            }
+          }
+          if (!ok) break;
+          umma_commit(bar(C::B_SFULL + (j & 1)));
+        }
+        if (j >= 1) {
+          const int i = j - 1;
+          PA_TRACE_ONLY(const long long tw = clock64();)
+          ok = thread_wait(bar(C::B_PFULL + (i & 1)), (i >> 1) & 1, abort_flag, tmo);
+          PA_TRACE_ONLY(const long long tv = clock64(); tr[1] += tv - tw; tlog(1, tln, 5, i);)
+          const uint32_t vslot0 = slot;  // the V tile takes slots vslot0, vslot0 + 1, ... (mod NSLOT)
+#pragma unroll
+          for (int k = 0; k < NP; ++k) {
+            if (ok) ok = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
+            if (++slot == (uint32_t)NSLOT) {
+              slot = 0;
+              ++round;
+            }
+          }
+          if (!ok) break;
+          PA_TRACE_ONLY(tlog(1, tln, 6, i);)
+          tc_fence_after();
+          const uint32_t p_tmem = tmem + kSCol0 + 128u * (i & 1) + kPColOff;
+#pragma unroll
+          for (int ks = 0; ks < kTileKeys / 16; ++ks) {
+            const uint32_t off = v_offset<NP, C::PANEL_LOG>(16u * ks, 0, a.v_shift);
+            uint32_t vs = vslot0 + (off >> 14);
+            if (vs >= (uint32_t)NSLOT) vs -= NSLOT;
+            umma_ts(tmem + kOCol, p_tmem + ks * 8,
+                    v_desc + vs * kSlotDesc + ((off & (kPanel - 1)) >> 4), idesc_pv,
+                    (i > 0 || ks > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < NP; ++k) {
+            uint32_t vs = vslot0 + k;
+            if (vs >= (uint32_t)NSLOT) vs -= NSLOT;
+            umma_commit(bar(C::B_EMPTY + vs));
+          }
+          umma_commit(bar(C::B_PVDONE));
+          PA_TRACE_ONLY(tr[2] += clock64() - tv; tlog(1, tln, 7, i);)
+        }
+      }
+      // Every issued MMA must finish before tensor memory is freed.
+      umma_commit(bar(C::B_MMADONE));
+      drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
+      PA_TRACE_ONLY(atomicAdd(&g_pa_trace[0], (unsigned long long)tr[0]);
+                    atomicAdd(&g_pa_trace[1], (unsigned long long)tr[1]);
+                    atomicAdd(&g_pa_trace[2], (unsigned long long)tr[2]);
+                    atomicAdd(&g_pa_trace[3], (unsigned long long)(clock64() - t_begin));)
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -560,10 +679,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// K or V as a 3-D tensor {D, Hkv, rows}; a box is 64 elements (128 B, one swizzle row) of
-// one KV head for `box_rows` consecutive key rows.
-bool make_kv_map(CUtensorMap* map, const void* base, bool bf16, int D, int Hkv, int64_t rows,
-                 int box_rows) {
+// K as a 3-D tensor {D, Hkv, rows}: a box is 64 elements (128 B, one swizzle row) of one KV
+// head for `box_rows` consecutive key rows.
+bool make_k_map(CUtensorMap* map, const void* base, bool bf16, int D, int Hkv, int64_t rows,
+                int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
@@ -572,6 +691,25 @@ bool make_kv_map(CUtensorMap* map, const void* base, bool bf16, int D, int Hkv, 
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r =
       fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// V as a 4-D tensor {64, rows, D/64 panels, Hkv}: a box is `panels` 64-wide panels of one KV
+// head for `box_rows` key rows, laid out panel after panel in shared memory (each panel a
+// column of 128-byte swizzled rows), which is the MN-major operand layout of P V.
+bool make_v_map(CUtensorMap* map, const void* base, bool bf16, int D, int Hkv, int64_t rows,
+                int box_rows, int panels) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)(D / 64), (cuuint64_t)Hkv};
+  const cuuint64_t strides[3] = {(cuuint64_t)Hkv * D * 2, 128, (cuuint64_t)D * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)panels, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r =
+      fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -647,9 +785,10 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
 
   CUtensorMap tk, tv;
   const int64_t rows = paged ? num_pages * PS : total_keys;
-  const int box_rows = paged ? PS : kTileKeys;
-  if (!make_kv_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, box_rows) ||
-      !make_kv_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, box_rows))
+  const int page_rows = paged ? PS : kTileKeys;            // key rows of one page (a K box)
+  const int v_rows = std::min(page_rows, 128 / (D / 64));   // a V box (all D) is <= 16 KB
+  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, page_rows) ||
+      !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, D / 64))
     return PA_ERR_CUDA;
 
   PrefillArgs a;
@@ -667,8 +806,11 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.G = plan->group;
   a.q_tiles = plan->q_tiles;
   a.splits = S;
-  a.page_size = paged ? PS : 0;
-  a.pages_per_tile = paged ? kTileKeys / PS : 1;
+  a.page_rows = page_rows;
+  a.page_shift = __builtin_ctz((unsigned)page_rows);
+  a.pages_per_tile = kTileKeys / page_rows;
+  a.v_rows = v_rows;
+  a.v_shift = __builtin_ctz((unsigned)v_rows);
   a.num_pages = paged ? (int32_t)num_pages : 0;
   a.oob_row = (int32_t)rows;
   a.scale_log2 = plan->scale * 1.4426950408889634f;
@@ -716,6 +858,31 @@ extern "C" int pa_device_error(int* flags, int reset) {
   if (v & kFlagTimeout) return PA_ERR_TIMEOUT;
   return PA_OK;
 }
+
+#ifdef PA_TRACE
+extern "C" int pa_trace_log(unsigned long long* out, int cap, int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  int n = cap < kLogCap ? cap : kLogCap;
+  if (cudaMemcpyFromSymbol(out, g_pa_log, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
+  if (reset) {
+    static unsigned long long z[kLogCap];
+    cudaMemcpyToSymbol(g_pa_log, z, sizeof z);
+  }
+  return n;
+}
+// Instrumented builds only: copy (and optionally clear) the kernel's cycle counters.
+extern "C" int pa_trace_read(unsigned long long* out, int n, int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+  if (n > 16) n = 16;
+  if (cudaMemcpyFromSymbol(out, g_pa_trace, n * sizeof(unsigned long long)) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (reset) {
+    unsigned long long z[16] = {0};
+    if (cudaMemcpyToSymbol(g_pa_trace, z, sizeof z) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+#endif
 
 extern "C" void pa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : 1); }
 

@@ -74,6 +74,27 @@ def test_ragged_full(idx):
         assert np.array_equal(a, b)
 
 
+MULTI_TILE = [
+    # a single unit spanning 2-3 KV tiles, and many units with 1-2 KV tiles (head dim 256)
+    (8, 1, 256, 16, "f16", [(200, 16)], 1),
+    (8, 1, 256, 16, "f16", [(300, 16)], 1),
+    (8, 1, 256, 64, "bf16", [(0, 256)], 1),
+    (8, 1, 256, 128, "f16", [(0, 256)], 1),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(MULTI_TILE)), ids=[f"m{i}" for i in range(len(MULTI_TILE))])
+def test_units_spanning_several_kv_tiles(idx):
+    """Every PV group must be complete before O is rescaled or read (the softmax tracks the
+    PV completions one by one); a unit with several KV tiles exercises that ordering."""
+    Hq, Hkv, D, PS, dt, pieces, S = MULTI_TILE[idx]
+    wl = U.custom_workload("multi", Hq, Hkv, D, PS, dt, pieces, seed=900 + idx, splits=S)
+    inp = U.gen(wl)
+    for paged in (True, False):
+        _, outs = U.run_gpu(inp, paged=paged)
+        U.check_full(inp, outs, paged=paged, what=f"{MULTI_TILE[idx]} paged={paged}")
+
+
 def test_online_rescale_with_growing_scores():
     wl = U.custom_workload("ramp", 16, 4, 256, 16, "bf16", [(1200, 160)], seed=77, splits=2)
     inp = U.gen(wl, distribution="ramp")
