@@ -143,6 +143,32 @@ int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_pool, const v
 int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes, float* out,
                pa_stream_t stream);
 
+/* Bytes of the device-resident scratch used by pa_prefill_noalloc (64 MiB). */
+#define PA_NOALLOC_WS_BYTES (64ull << 20)
+
+/*
+ * pa_prefill_noalloc — pa_prefill followed by pa_combine, for callers that cannot allocate
+ * device memory: for example a plugin inside a serving engine that has reserved all device
+ * memory for its KV-cache pool and exposes no allocator, or a caller that cannot afford the
+ * implicit device synchronisation an allocation may cause. (The pages describe no such entry
+ * point; it has no counterpart there.)
+ *   Arguments are those of pa_prefill, without lse_ws / ws_bytes: when plan->splits > 1 the
+ *   split partials go to a scratch array that the library holds in device memory on every
+ *   device it is loaded on (PA_NOALLOC_WS_BYTES, kept until the process exits). out is
+ *   written in full, as pa_prefill + pa_combine would write it.
+ *   The first call on a device looks the scratch's device address up (a runtime call, made
+ *   with that device current); make that first call before any stream capture.
+ *   Every call shares the one scratch array, which keeps the last call's contents (nothing in
+ *   it needs to start at zero: each call writes every entry it reads). Calls whose work may
+ *   overlap on the GPU (different streams, or several host threads without ordering) race on
+ *   it: order them, e.g. issue them on one stream.
+ * Returns PA_ERR_WORKSPACE when plan->ws_bytes exceeds PA_NOALLOC_WS_BYTES, else what
+ * pa_prefill / pa_combine return. Allocates nothing (no cudaMalloc, no cudaFree).
+ */
+int pa_prefill_noalloc(const pa_plan_t* plan, const void* q, const void* k_pool,
+                       const void* v_pool, const int32_t* page_table, int64_t num_pages,
+                       int64_t hist_len, int chunk_rows, float* out, pa_stream_t stream);
+
 /*
  * pa_device_error — synchronise the current device, then read (and with reset != 0,
  * clear) the library's device-side error word. *flags receives its bits

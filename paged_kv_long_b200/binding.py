@@ -18,7 +18,8 @@ PA_F16, PA_BF16 = 0, 1
 POLICIES = {"makespan": 0, "cores": 1, "legacy": 2}
 STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
           -4: "PA_ERR_CUDA", -5: "PA_ERR_TIMEOUT", -6: "PA_ERR_PAGE_INDEX"}
-EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_device_error", "pa_set_wait_timeout_ns",
+EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_device_error",
+            "pa_set_wait_timeout_ns",
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
             "pa_legacy_policy_splits")
 
@@ -68,6 +69,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_prefill.restype = i32
     lib.pa_combine.argtypes = [ctypes.POINTER(Plan), vp, u64, vp, vp]
     lib.pa_combine.restype = i32
+    lib.pa_prefill_noalloc.argtypes = [ctypes.POINTER(Plan), vp, vp, vp, vp, i64, i64, i32, vp, vp]
+    lib.pa_prefill_noalloc.restype = i32
     lib.pa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), i32]
     lib.pa_device_error.restype = i32
     lib.pa_set_wait_timeout_ns.argtypes = [u64]
@@ -201,6 +204,27 @@ def prefill_combine(p: Plan, q, k_pool, v_pool, page_table, out=None, ws=None, s
     prefill(p, q, k_pool, v_pool, page_table, out, ws, stream)
     combine(p, ws, out, stream)
     return out
+
+
+def prefill_noalloc(p: Plan, q, k_pool, v_pool, page_table, out, stream=None):
+    """pa_prefill_noalloc: prefill + combine with the library's own device scratch (for
+    callers that cannot allocate device memory; see include/pa.h)."""
+    import torch
+    dt = _torch_dtype(p)
+    R, Hq, D = p.chunk_rows, p.n_q_heads, p.head_dim
+    _require_cuda(q, "q", dt, (R, Hq, D))
+    _require_cuda(k_pool, "k_pool", dt)
+    _require_cuda(v_pool, "v_pool", dt, tuple(k_pool.shape))
+    _require_cuda(out, "out", torch.float32, (R, Hq, D))
+    if p.paged:
+        _require_cuda(page_table, "page_table", torch.int32)
+        num_pages, tab = k_pool.shape[0], page_table.data_ptr()
+    else:
+        num_pages, tab = 0, None
+    st = load_library().pa_prefill_noalloc(ctypes.byref(p), q.data_ptr(), k_pool.data_ptr(),
+                                           v_pool.data_ptr(), tab, num_pages, p.hist_len, R,
+                                           out.data_ptr(), _stream_ptr(stream))
+    _check(st, "pa_prefill_noalloc")
 
 
 def device_error(reset: bool = True) -> tuple[int, int]:

@@ -844,6 +844,49 @@ extern "C" int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t w
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- entry point without allocation
+// Scratch of pa_prefill_noalloc: the split partials and their log-sum-exps live in this
+// file-scope device array (every device that loads the library holds it until exit), so the
+// entry point needs no allocation at all. Host code may not pass the symbol itself to a
+// kernel (on the host it is only a stand-in, not a device address): its device address is
+// looked up once per device with cudaGetSymbolAddress, with that device current.
+static __device__ __align__(256) float g_noalloc_ws[PA_NOALLOC_WS_BYTES / sizeof(float)];
+static std::mutex g_noalloc_mu;
+static float* g_noalloc_ptr[64];  // per device ordinal; null until its first call
+
+static int noalloc_scratch(float** ws) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return PA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) return PA_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *ws = g_noalloc_ptr[dev];
+  return PA_OK;
+}
+
+extern "C" int pa_prefill_noalloc(const pa_plan_t* plan, const void* q, const void* k_pool,
+                                  const void* v_pool, const int32_t* page_table, int64_t num_pages,
+                                  int64_t hist_len, int chunk_rows, float* out,
+                                  pa_stream_t stream) {
+  if (!plan) return PA_ERR_INVALID_ARG;
+  float* ws = nullptr;
+  uint64_t ws_bytes = 0;
+  if (plan->splits > 1) {
+    if (plan->ws_bytes > PA_NOALLOC_WS_BYTES) return PA_ERR_WORKSPACE;
+    const int st = noalloc_scratch(&ws);
+    if (st != PA_OK) return st;
+    ws_bytes = PA_NOALLOC_WS_BYTES;
+  }
+  const int st = pa_prefill(plan, q, k_pool, v_pool, page_table, num_pages, hist_len, chunk_rows,
+                            out, ws, ws_bytes, stream);
+  if (st != PA_OK) return st;
+  return pa_combine(plan, ws, ws_bytes, out, stream);
+}
+
 extern "C" int pa_device_error(int* flags, int reset) {
   if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
   unsigned v = 0;
