@@ -72,7 +72,9 @@ typedef enum {
  * r of KV head g is token r / G, Q head g*G + r % G. A Q tile is PA_TILE_ROWS consecutive
  * packed rows (a tile may start inside a token's head group). Work units are
  * (KV head, Q tile, split); split s of a tile whose tokens end at t_last covers KV tiles
- * [s*n/S, (s+1)*n/S) of the n = ceil((H + t_last + 1) / PA_TILE_KEYS) tiles it sees.
+ * [s*n/S, (s+1)*n/S) of the n = ceil((H + t_last + 1) / PA_TILE_KEYS) tiles it sees. With
+ * ctas_per_unit = 2 a unit is a pair of consecutive Q tiles (2t, 2t+1) on a CTA pair, and t_last
+ * is that of the pair's last tile.
  */
 typedef struct {
   int32_t num_sms;        /* SMs the plan was made for */
@@ -87,8 +89,10 @@ typedef struct {
   int32_t paged;          /* 1: k/v are page pools read through page_table; 0: contiguous */
   int32_t dtype;          /* pa_dtype of q, k, v */
   int32_t policy;         /* pa_policy used (or -1 when splits was overridden) */
+  int32_t ctas_per_unit;  /* 2: head_dim 256 runs on CTA pairs (two Q tiles per unit); else 1 */
+  int32_t reserved;
   int64_t hist_len;       /* H: keys in the cache before the piece */
-  int64_t units;          /* Hkv * q_tiles * S CTAs of the prefill kernel */
+  int64_t units;          /* Hkv * ceil(q_tiles / ctas_per_unit) * S units (CTAs or pairs) */
   float scale;            /* softmax scale actually used */
   float est_us;           /* the planner's time estimate for prefill + combine (microseconds) */
   uint64_t ws_bytes;      /* bytes of lse_ws needed: S*R*Hq*(D+1)*4 if S > 1, else 0 */

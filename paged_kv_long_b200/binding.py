@@ -37,7 +37,7 @@ class Plan(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("group", ctypes.c_int32),
         ("chunk_rows", ctypes.c_int32), ("q_tiles", ctypes.c_int32), ("splits", ctypes.c_int32),
         ("paged", ctypes.c_int32), ("dtype", ctypes.c_int32), ("policy", ctypes.c_int32),
-        ("hist_len", ctypes.c_int64), ("units", ctypes.c_int64), ("scale", ctypes.c_float),
+        ("ctas_per_unit", ctypes.c_int32), ("reserved", ctypes.c_int32), ("hist_len", ctypes.c_int64), ("units", ctypes.c_int64), ("scale", ctypes.c_float),
         ("est_us", ctypes.c_float), ("ws_bytes", ctypes.c_uint64),
     ]
 

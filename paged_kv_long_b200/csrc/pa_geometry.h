@@ -45,6 +45,15 @@ PA_HD void split_range(int64_t n_kt, int s, int S, int64_t* kt0, int64_t* kt1) {
   *kt1 = (int64_t)(s + 1) * n_kt / S;
 }
 
+// KV tiles visible to unit-tile qu, when a unit covers `per_unit` consecutive Q tiles (1 or
+// 2): those of its last Q tile.
+PA_HD int64_t unit_kv_tiles(int64_t qu, int per_unit, int64_t q_tiles, int64_t R, int G,
+                            int64_t H) {
+  int64_t last = qu * per_unit + per_unit - 1;
+  if (last > q_tiles - 1) last = q_tiles - 1;
+  return tile_kv_tiles(last, R, G, H);
+}
+
 // Unit u -> (Q tile, KV head, split). Units run longest first: the last Q tile (most keys)
 // gets the lowest unit indices.
 PA_HD void unit_coords(int64_t u, int64_t q_tiles, int Hkv, int S, int64_t* qt, int* g, int* s) {

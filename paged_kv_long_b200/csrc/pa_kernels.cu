@@ -64,6 +64,7 @@ struct PrefillArgs {
   int32_t page_rows;     // key rows per page: the page size, or kTileKeys when contiguous
   int32_t page_shift;    // log2(page_rows)
   int32_t pages_per_tile;
+  int32_t k_rows;        // key rows per K box (CTA-pair kernel: <= 64, half a tile)
   int32_t v_rows;        // key rows per V box (<= page_rows; a box is at most one slot)
   int32_t v_shift;       // log2(v_rows)
   int32_t num_pages;
@@ -85,10 +86,10 @@ struct Cfg {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = Q_OFF + NP * kPanel;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * kPanel;
-  // barriers: full[NSLOT], empty[NSLOT], q_full, s_full[2], p_full[2], pv_done, mma_done
+  // barriers: full[NSLOT], empty[NSLOT], q_full, s_full[2], p_full[2], pv_done[2], mma_done
   static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_QFULL = 2 * NSLOT, B_SFULL = 2 * NSLOT + 1,
                        B_PFULL = 2 * NSLOT + 3, B_PVDONE = 2 * NSLOT + 5,
-                       B_MMADONE = 2 * NSLOT + 6, N_BARS = 2 * NSLOT + 7;
+                       B_MMADONE = 2 * NSLOT + 7, N_BARS = 2 * NSLOT + 8;
   static constexpr int MISC_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int SMEM = MISC_OFF + 16;
   static constexpr int LAUNCH_SMEM = SMEM + 1024;    // slack to align the base to 1024 B
@@ -112,13 +113,14 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
 // Instrumented builds only: cycle counters summed over all CTAs (see pa_trace_read), and an
 // event log of the first CTAs: (kind << 56 | cta << 48 | index << 32 | clock low 32 bits).
 __device__ unsigned long long g_pa_trace[16];
-constexpr int kLogCap = 1 << 16;  // 2 CTAs x 3 roles x 8192 events
+constexpr int kLogCap = 1 << 16;  // 2 CTAs x 8 roles x 4096 events
 __device__ unsigned long long g_pa_log[kLogCap];
-// role: 0 producer, 1 MMA, 2 softmax; `n` is the role's own event counter (no atomics).
+// role: 0-2 TMA warps (or 0 the single producer), 1 MMA in the single-CTA kernel, 3 MMA,
+// 4 fill observer, 5 softmax; `n` is the role's own event counter (no atomics).
 __device__ __forceinline__ void tlog(int role, unsigned& n, int kind, int index) {
   const unsigned long long clk = (unsigned)clock64();
-  if (blockIdx.x < 2 && n < 8192u)
-    g_pa_log[(blockIdx.x * 3 + role) * 8192 + n++] =
+  if (blockIdx.x < 2 && n < 4096u)
+    g_pa_log[(blockIdx.x * 8 + role) * 4096 + n++] =
         ((unsigned long long)kind << 56) | ((unsigned long long)blockIdx.x << 48) |
         ((unsigned long long)(index & 0xFFFF) << 32) | clk;
 }
@@ -174,6 +176,211 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   }
 }
 
+// Softmax + epilogue warps (warps 0-3: one thread per packed Q row = tensor-memory lane), for
+// both kernels. The pair kernel's second CTA announces Q and P on the first CTA's barriers
+// (remote arrivals); everything else it reads and writes is its own.
+struct SoftmaxCtx {
+  uint32_t sb, q_off;
+  uint32_t bar_sfull, bar_pvdone;      // local barriers: S buffers 0/1, PV groups of even/odd tiles
+  uint32_t arrive_qfull, arrive_pfull; // where Q / P readiness is announced (maybe remote)
+  bool remote_arrive;
+  uint32_t tmem;
+  int64_t qt;
+  int g, s;
+  int64_t kt0;
+  int n;
+  volatile int* abort_flag;
+  uint64_t tmo;
+};
+
+template <int D, bool PAGED, bool BF16, class VTail>
+__device__ __forceinline__ void softmax_role(const PrefillArgs& a, const SoftmaxCtx& x,
+                                             VTail&& v_tail) {
+  constexpr int NP = D / 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sb = x.sb, tmem = x.tmem;
+  const int64_t qt = x.qt, kt0 = x.kt0;
+  const int g = x.g, s = x.s, n = x.n;
+  volatile int* abort_flag = x.abort_flag;
+  const uint64_t tmo = x.tmo;
+  auto arrive = [&](uint32_t addr) {
+    if (x.remote_arrive)
+      mbar_arrive_remote(addr);
+    else
+      mbar_arrive(addr);
+  };
+  PA_TRACE_ONLY(long long tr[4] = {0, 0, 0, 0}; const long long t_begin = clock64(); unsigned tln = 0;)
+  {
+    const int r = threadIdx.x;  // packed Q row = tensor-memory lane
+    const int64_t grow = qt * kTileRows + r;
+    const int64_t tok = grow / a.G;
+    const bool valid = tok < a.R;
+    const int head = g * a.G + (int)(grow % a.G);
+    {
+      // Q tile -> shared memory as K-major rows of 64-element panels, 128-byte swizzle.
+      const uint4* src =
+          reinterpret_cast<const uint4*>(a.q + (valid ? (tok * a.Hq + head) * (int64_t)D : 0));
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = valid ? __ldg(src + p * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+          st_shared_v4(sb + x.q_off + p * kPanel + r * 128 + ((c ^ (r & 7)) << 4), v.x, v.y, v.z,
+                       v.w);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) arrive(x.arrive_qfull);
+    }
+
+    const int64_t limit = valid ? a.hist_len + tok : -1;  // last key this row may see
+    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    float m_run = -INFINITY;  // running max of scale*log2(e)*score
+    float l_run = 0.f;        // running sum of the probabilities (fp32)
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int sbuf = j & 1;
+      const uint32_t s_col = kSCol0 + 128u * sbuf;
+      const int64_t key0 = (kt0 + j) * kTileKeys;
+      PA_TRACE_ONLY(long long tw = clock64();)
+      if (!warp_wait(x.bar_sfull + 8u * sbuf, (j >> 1) & 1, abort_flag, tmo)) {
+        ok = false;
+        break;
+      }
+      PA_TRACE_ONLY(const long long tc = clock64(); tr[0] += tc - tw;
+                    if (threadIdx.x == 0) tlog(5, tln, 8, j);)
+      tc_fence_after();
+      float sv[kTileKeys];
+#pragma unroll
+      for (int c = 0; c < kTileKeys / 32; ++c)
+        tmem_ld32(t_lane + s_col + 32u * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
+      tmem_wait_ld();
+
+      // causal mask by select (masked scores become -inf, whatever bits they held)
+      const int64_t rel64 = limit - key0;
+      if (rel64 < kTileKeys - 1) {
+        const int rel = rel64 < -1 ? -1 : (int)rel64;
+#pragma unroll
+        for (int c = 0; c < kTileKeys; ++c)
+          if (c > rel) sv[c] = -INFINITY;
+      }
+      // row max: eight independent chains, then a tree
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+#pragma unroll
+      for (int c = 8; c < kTileKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_new = fmaxf(m_run, mx * a.scale_log2);
+      const bool need = m_new > m_run + kRescaleLog2;
+      // PV of tile i completes phase i/2 of pv_done[i % 2]. Parity waits are sound only if no
+      // phase is skipped: the softmax observes PV_{j-2} before it releases P_j (PV_j, the next
+      // completion on that barrier, cannot happen earlier), and PV_{j-1} only when O must be
+      // rescaled. P_j thus never waits for the PV just before it.
+      if (j == 0) {
+        if (need) m_run = m_new;
+      } else if (__any_sync(0xffffffffu, need)) {
+        // O must not change under a running MMA: wait for PV of the previous tile.
+        if (!warp_wait(x.bar_pvdone + 8u * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = need ? ex2(m_run - m_new) : 1.0f;
+        l_run *= f;
+        PA_TRACE_ONLY(tr[3] += 1;)
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(t_lane + kOCol + 32u * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= f;
+          tmem_st32(t_lane + kOCol + 32u * c, o);
+        }
+        tmem_wait_st();
+        if (need) m_run = m_new;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // two 64-key halves -> 32 columns of P each
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 x = ffma2(make_float2(sv[64 * h + c], sv[64 * h + c + 1]), sc2, nm2);
+          const float2 pr = make_float2(ex2(x.x), ex2(x.y));
+          ls[(c >> 1) & 3] = fadd2(ls[(c >> 1) & 3], pr);
+          pk[c >> 1] = pack2<BF16>(pr.x, pr.y);
+        }
+        tmem_st32u(t_lane + s_col + kPColOff + 32u * h, pk);
+      }
+      l_run += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y) + (ls[2].x + ls[2].y) +
+               (ls[3].x + ls[3].y);
+      if (j >= 2 && !warp_wait(x.bar_pvdone + 8u * (j & 1), ((j - 2) >> 1) & 1, abort_flag, tmo)) {
+        ok = false;
+        break;
+      }
+
+      if constexpr (PAGED) {
+        if (key0 + kTileKeys > a.total_keys) {
+          const bool zero_me = key0 + r >= a.total_keys;
+          if (!v_tail(j, zero_me ? r : -1)) {
+            ok = false;
+            break;
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive(x.arrive_pfull + 8u * sbuf);
+      PA_TRACE_ONLY(tr[1] += clock64() - tc; if (threadIdx.x == 0) tlog(5, tln, 9, j);)
+    }
+
+    PA_TRACE_ONLY(const long long te = clock64();)
+    if (ok && n >= 2)
+      ok = warp_wait(x.bar_pvdone + 8u * ((n - 2) & 1), ((n - 2) >> 1) & 1, abort_flag, tmo);
+    if (ok) ok = warp_wait(x.bar_pvdone + 8u * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, tmo);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      float* dst = (a.splits == 1) ? a.out + (tok * a.Hq + head) * (int64_t)D
+                                   : a.ws_o + (((int64_t)s * a.R + tok) * a.Hq + head) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(t_lane + kOCol + 32u * c, o);
+        tmem_wait_ld();
+        if (valid) {
+          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d4[i] = make_float4(o[4 * i] * inv_l, o[4 * i + 1] * inv_l, o[4 * i + 2] * inv_l,
+                                o[4 * i + 3] * inv_l);
+        }
+      }
+      if (valid && a.splits > 1)
+        a.ws_lse[((int64_t)s * a.R + tok) * a.Hq + head] =
+            l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+    }
+    PA_TRACE_ONLY(tr[2] += clock64() - te;
+                  if (lane == 0) {
+                    atomicAdd(&g_pa_trace[6], (unsigned long long)tr[0]);
+                    atomicAdd(&g_pa_trace[7], (unsigned long long)tr[1]);
+                    atomicAdd(&g_pa_trace[8], (unsigned long long)tr[2]);
+                    atomicAdd(&g_pa_trace[9], (unsigned long long)tr[3]);
+                    atomicAdd(&g_pa_trace[10], (unsigned long long)(clock64() - t_begin));
+                    if (warp == 0) atomicAdd(&g_pa_trace[11], (unsigned long long)n);
+                  })
+  }
+}
+
 // ---------------------------------------------------------------- prefill kernel
 template <int D, bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -225,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(C::B_SFULL + 1), 1);
     mbar_init(bar(C::B_PFULL + 0), 4);
     mbar_init(bar(C::B_PFULL + 1), 4);
-    mbar_init(bar(C::B_PVDONE), 1);
+    mbar_init(bar(C::B_PVDONE + 0), 1);
+    mbar_init(bar(C::B_PVDONE + 1), 1);
     mbar_init(bar(C::B_MMADONE), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -248,187 +456,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     // ============================================================ softmax + epilogue
-    const int r = threadIdx.x;  // packed Q row = tensor-memory lane
-    const int64_t grow = qt * kTileRows + r;
-    const int64_t tok = grow / a.G;
-    const bool valid = tok < a.R;
-    const int head = g * a.G + (int)(grow % a.G);
-    {
-      // Q tile -> shared memory as K-major rows of 64-element panels, 128-byte swizzle.
-      const uint4* src =
-          reinterpret_cast<const uint4*>(a.q + (valid ? (tok * a.Hq + head) * (int64_t)D : 0));
-#pragma unroll
+    SoftmaxCtx sc;
+    sc.sb = sb;
+    sc.q_off = C::Q_OFF;
+    sc.bar_sfull = bar(C::B_SFULL);
+    sc.bar_pvdone = bar(C::B_PVDONE);
+    sc.arrive_qfull = bar(C::B_QFULL);
+    sc.arrive_pfull = bar(C::B_PFULL);
+    sc.remote_arrive = false;
+    sc.tmem = tmem;
+    sc.qt = qt;
+    sc.g = g;
+    sc.s = s;
+    sc.kt0 = kt0;
+    sc.n = n;
+    sc.abort_flag = abort_flag;
+    sc.tmo = tmo;
+    // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
+    // is NaN inside the MMA, so those V rows are zeroed before PV reads them.
+    auto v_tail = [&](int j, int r) -> bool {
+      const uint32_t seq0 = v_item(j, n) * NP;
+      bool okv = true;
+      for (int p = 0; p < NP && okv; ++p)
+        okv = warp_wait(bar(C::B_FULL + (seq0 + p) % NSLOT), ((seq0 + p) / NSLOT) & 1, abort_flag,
+                        tmo);
+      if (!okv || r < 0) return okv;
       for (int p = 0; p < NP; ++p) {
+        const uint32_t off = v_offset<NP, C::PANEL_LOG>((uint32_t)r, p, a.v_shift);
+        const uint32_t ra = slot_addr((seq0 + (off >> 14)) % NSLOT) + (off & (kPanel - 1));
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = valid ? __ldg(src + p * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
-          st_shared_v4(sb + C::Q_OFF + p * kPanel + r * 128 + ((c ^ (r & 7)) << 4), v.x, v.y, v.z,
-                       v.w);
-        }
+        for (int c = 0; c < 8; ++c) st_shared_v4(ra + c * 16, 0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_QFULL));
-    }
-
-    const int64_t limit = valid ? a.hist_len + tok : -1;  // last key this row may see
-    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
-    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-    float m_run = -INFINITY;  // running max of scale*log2(e)*score
-    float l_run = 0.f;        // running sum of the probabilities (fp32)
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int sbuf = j & 1;
-      const uint32_t s_col = kSCol0 + 128u * sbuf;
-      const int64_t key0 = (kt0 + j) * kTileKeys;
-      PA_TRACE_ONLY(long long tw = clock64();)
-      if (!warp_wait(bar(C::B_SFULL + sbuf), (j >> 1) & 1, abort_flag, tmo)) {
-        ok = false;
-        break;
-      }
-      PA_TRACE_ONLY(const long long tc = clock64(); tr[0] += tc - tw;
-                    if (threadIdx.x == 0) tlog(2, tln, 8, j);)
-      tc_fence_after();
-      float sv[kTileKeys];
-#pragma unroll
-      for (int c = 0; c < kTileKeys / 32; ++c)
-        tmem_ld32(t_lane + s_col + 32u * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
-      tmem_wait_ld();
-
-      // causal mask by select (masked scores become -inf, whatever bits they held)
-      const int64_t rel64 = limit - key0;
-      if (rel64 < kTileKeys - 1) {
-        const int rel = rel64 < -1 ? -1 : (int)rel64;
-#pragma unroll
-        for (int c = 0; c < kTileKeys; ++c)
-          if (c > rel) sv[c] = -INFINITY;
-      }
-      // row max: eight independent chains, then a tree
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
-#pragma unroll
-      for (int c = 8; c < kTileKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_new = fmaxf(m_run, mx * a.scale_log2);
-      const bool need = m_new > m_run + kRescaleLog2;
-      // pv_done completes once per PV MMA group, in order. Parity waits are only sound when
-      // no phase is skipped, so every tile j >= 1 observes PV_{j-1} before it releases P_j
-      // (PV_j cannot finish before that); here early when O must be rescaled, else below.
-      bool pv_prev_seen = (j == 0);
-      if (j == 0) {
-        if (need) m_run = m_new;
-      } else if (__any_sync(0xffffffffu, need)) {
-        // O must not change under a running MMA: wait for PV of the previous tile.
-        if (!warp_wait(bar(C::B_PVDONE), (j - 1) & 1, abort_flag, tmo)) {
-          ok = false;
-          break;
-        }
-        pv_prev_seen = true;
-        tc_fence_after();
-        const float f = need ? ex2(m_run - m_new) : 1.0f;
-        l_run *= f;
-        PA_TRACE_ONLY(tr[3] += 1;)
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(t_lane + kOCol + 32u * c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= f;
-          tmem_st32(t_lane + kOCol + 32u * c, o);
-        }
-        tmem_wait_st();
-        if (need) m_run = m_new;
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      const float2 nm2 = make_float2(-m_use, -m_use);
-      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                      make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {  // two 64-key halves -> 32 columns of P each
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float2 x = ffma2(make_float2(sv[64 * h + c], sv[64 * h + c + 1]), sc2, nm2);
-          const float2 pr = make_float2(ex2(x.x), ex2(x.y));
-          ls[(c >> 1) & 3] = fadd2(ls[(c >> 1) & 3], pr);
-          pk[c >> 1] = pack2<BF16>(pr.x, pr.y);
-        }
-        tmem_st32u(t_lane + s_col + kPColOff + 32u * h, pk);
-      }
-      l_run += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y) + (ls[2].x + ls[2].y) +
-               (ls[3].x + ls[3].y);
-      if (!pv_prev_seen && !warp_wait(bar(C::B_PVDONE), (j - 1) & 1, abort_flag, tmo)) {
-        ok = false;
-        break;
-      }
-
-      if constexpr (PAGED) {
-        // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but
-        // 0 * NaN is NaN inside the MMA, so those V rows are zeroed before PV reads them.
-        if (key0 + kTileKeys > a.total_keys) {
-          const uint32_t seq0 = v_item(j, n) * NP;
-          bool okv = true;
-          for (int p = 0; p < NP && okv; ++p)
-            okv = warp_wait(bar(C::B_FULL + (seq0 + p) % NSLOT), ((seq0 + p) / NSLOT) & 1,
-                            abort_flag, tmo);
-          if (!okv) {
-            ok = false;
-            break;
-          }
-          if (key0 + r >= a.total_keys) {
-            for (int p = 0; p < NP; ++p) {
-              const uint32_t off = v_offset<NP, C::PANEL_LOG>((uint32_t)r, p, a.v_shift);
-              const uint32_t ra = slot_addr((seq0 + (off >> 14)) % NSLOT) + (off & (kPanel - 1));
-#pragma unroll
-              for (int c = 0; c < 8; ++c) st_shared_v4(ra + c * 16, 0u, 0u, 0u, 0u);
-            }
-            fence_proxy_async_smem();
-          }
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_PFULL + sbuf));
-      PA_TRACE_ONLY(tr[1] += clock64() - tc; if (threadIdx.x == 0) tlog(2, tln, 9, j);)
-    }
-
-    PA_TRACE_ONLY(const long long te = clock64();)
-    if (ok) ok = warp_wait(bar(C::B_PVDONE), (n - 1) & 1, abort_flag, tmo);
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      float* dst = (a.splits == 1) ? a.out + (tok * a.Hq + head) * (int64_t)D
-                                   : a.ws_o + (((int64_t)s * a.R + tok) * a.Hq + head) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(t_lane + kOCol + 32u * c, o);
-        tmem_wait_ld();
-        if (valid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(o[4 * i] * inv_l, o[4 * i + 1] * inv_l, o[4 * i + 2] * inv_l,
-                                o[4 * i + 3] * inv_l);
-        }
-      }
-      if (valid && a.splits > 1)
-        a.ws_lse[((int64_t)s * a.R + tok) * a.Hq + head] =
-            l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
-    }
-    PA_TRACE_ONLY(tr[2] += clock64() - te;
-                  if (lane == 0) {
-                    atomicAdd(&g_pa_trace[6], (unsigned long long)tr[0]);
-                    atomicAdd(&g_pa_trace[7], (unsigned long long)tr[1]);
-                    atomicAdd(&g_pa_trace[8], (unsigned long long)tr[2]);
-                    atomicAdd(&g_pa_trace[9], (unsigned long long)tr[3]);
-                    atomicAdd(&g_pa_trace[10], (unsigned long long)(clock64() - t_begin));
-                    if (warp == 0) atomicAdd(&g_pa_trace[11], (unsigned long long)n);
-                  })
+      return true;
+    };
+    softmax_role<D, PAGED, BF16>(a, sc, v_tail);
   } else if (warp > kMmaWarp) {
     // ============================================================ TMA issuers (three warps)
     const int w = warp - kMmaWarp - 1;  // this warp issues fill numbers q with q % kIssuers == w
@@ -589,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (vs >= (uint32_t)NSLOT) vs -= NSLOT;
             umma_commit(bar(C::B_EMPTY + vs));
           }
-          umma_commit(bar(C::B_PVDONE));
+          umma_commit(bar(C::B_PVDONE + (i & 1)));
           PA_TRACE_ONLY(tr[2] += clock64() - tv; tlog(1, tln, 7, i);)
         }
       }
@@ -611,6 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
 }
+
+#include "prefill_pair.cuh"
 
 // ---------------------------------------------------------------- combine kernel
 // One warp per (row, head): lanes hold the S <= 32 split LSEs, the warp reduces max and sum
@@ -735,6 +799,38 @@ cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
   return cudaGetLastError();
 }
 
+template <bool PAGED, bool BF16>
+cudaError_t launch_pair(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
+                        const CUtensorMap& tv, const PrefillArgs& a) {
+  auto kern = prefill_pair_kernel<PAGED, BF16>;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairCfg::LAUNCH_SMEM);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg::LAUNCH_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_d(bool paged, bool bf16, int64_t grid, cudaStream_t st, const CUtensorMap& tk,
                      const CUtensorMap& tv, const PrefillArgs& a) {
@@ -778,17 +874,23 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
     if (!page_table || num_pages <= 0) return PA_ERR_INVALID_ARG;
     if (num_pages * PS + kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   }
-  const int64_t grid = plan->units;
-  if (grid != (int64_t)plan->q_tiles * plan->n_kv_heads * S || grid <= 0 ||
-      grid >= (int64_t(1) << 31))
+  const int per = plan->ctas_per_unit;
+  if (per != (D == 256 ? 2 : 1)) return PA_ERR_INVALID_ARG;
+  const int64_t q_units = ((int64_t)plan->q_tiles + per - 1) / per;
+  const int64_t grid = plan->units * per;  // CTAs
+  if (plan->units != q_units * plan->n_kv_heads * S || grid <= 0 || grid >= (int64_t(1) << 31))
     return PA_ERR_INVALID_ARG;
 
   CUtensorMap tk, tv;
   const int64_t rows = paged ? num_pages * PS : total_keys;
-  const int page_rows = paged ? PS : kTileKeys;            // key rows of one page (a K box)
-  const int v_rows = std::min(page_rows, 128 / (D / 64));   // a V box (all D) is <= 16 KB
-  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, page_rows) ||
-      !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, D / 64))
+  const int page_rows = paged ? PS : kTileKeys;  // key rows of one page
+  // Single CTA: a K box is a page (one 64-wide panel), a V box covers all of D (<= 16 KB).
+  // CTA pair: each CTA loads 64 keys of K and half of D of V, in boxes of <= 64 keys.
+  const int k_rows = per == 2 ? std::min(page_rows, 64) : page_rows;
+  const int v_rows = per == 2 ? std::min(page_rows, 64) : std::min(page_rows, 128 / (D / 64));
+  const int v_panels = per == 2 ? 2 : D / 64;
+  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows) ||
+      !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, v_panels))
     return PA_ERR_CUDA;
 
   PrefillArgs a;
@@ -809,6 +911,7 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.page_rows = page_rows;
   a.page_shift = __builtin_ctz((unsigned)page_rows);
   a.pages_per_tile = kTileKeys / page_rows;
+  a.k_rows = k_rows;
   a.v_rows = v_rows;
   a.v_shift = __builtin_ctz((unsigned)v_rows);
   a.num_pages = paged ? (int32_t)num_pages : 0;
@@ -821,7 +924,12 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   switch (D) {
     case 64: e = launch_d<64>(paged, bf16, grid, st, tk, tv, a); break;
     case 128: e = launch_d<128>(paged, bf16, grid, st, tk, tv, a); break;
-    default: e = launch_d<256>(paged, bf16, grid, st, tk, tv, a); break;
+    default:
+      e = paged ? (bf16 ? launch_pair<true, true>(grid, st, tk, tv, a)
+                        : launch_pair<true, false>(grid, st, tk, tv, a))
+                : (bf16 ? launch_pair<false, true>(grid, st, tk, tv, a)
+                        : launch_pair<false, false>(grid, st, tk, tv, a));
+      break;
   }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -38,15 +38,20 @@ struct CostModel {
   }
 };
 
+// CTAs per unit: head dim 256 runs on CTA pairs (two Q tiles share each K/V tile load).
+int ctas_per_unit_for(int D) { return D == 256 ? 2 : 1; }
+
 double simulate(int num_sms, int64_t q_tiles, int64_t R, int G, int Hkv, int64_t H, int S,
                 int D) {
   const CostModel cm(D);
+  const int per = ctas_per_unit_for(D);
+  const int64_t q_units = (q_tiles + per - 1) / per;
   std::priority_queue<double, std::vector<double>, std::greater<double>> sms;
-  for (int i = 0; i < num_sms; ++i) sms.push(0.0);
+  for (int i = 0; i < num_sms / per; ++i) sms.push(0.0);  // a pair unit holds two SMs
   double makespan = 0.0;
   // Units in launch order: last Q tile first; within a tile, KV heads then splits.
-  for (int64_t qt = q_tiles - 1; qt >= 0; --qt) {
-    const int64_t n_kt = pa::tile_kv_tiles(qt, R, G, H);
+  for (int64_t qt = q_units - 1; qt >= 0; --qt) {
+    const int64_t n_kt = pa::unit_kv_tiles(qt, per, q_tiles, R, G, H);
     for (int g = 0; g < Hkv; ++g) {
       for (int s = 0; s < S; ++s) {
         int64_t kt0, kt1;
@@ -104,8 +109,10 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
 
   const int G = n_q_heads / n_kv_heads;
   const int64_t q_tiles = pa::q_tiles_for(chunk_rows, G);
-  if (q_tiles * n_kv_heads * PA_MAX_SPLITS >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  if (q_tiles * n_kv_heads * PA_MAX_SPLITS * 2 >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   const int64_t max_kt = pa::tile_kv_tiles(q_tiles - 1, chunk_rows, G, hist_len);
+  const int per = ctas_per_unit_for(head_dim);
+  const int64_t q_units = (q_tiles + per - 1) / per;
 
   int S = 1;
   int used_policy = policy;
@@ -118,10 +125,10 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
     S = pa_legacy_policy_splits(n_kv_heads, (int)std::min<int64_t>(q_tiles, 1 << 30));
   } else {
     double best = 0.0;
-    const int64_t base_units = q_tiles * n_kv_heads;
+    const int64_t base_units = q_units * n_kv_heads;
     for (int cand = 1; cand <= PA_MAX_SPLITS; ++cand) {
       if (cand > 1 && cand > max_kt) break;                   // more splits than KV tiles
-      if (cand > 1 && base_units * cand > 16LL * num_sms) break;  // far past filling the GPU
+      if (cand > 1 && base_units * per * cand > 16LL * num_sms) break;  // far past full
       const double t = simulate(num_sms, q_tiles, chunk_rows, G, n_kv_heads, hist_len, cand,
                                 head_dim) +
                        combine_cost(cand, chunk_rows, n_q_heads, head_dim);
@@ -144,8 +151,10 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
   plan->paged = paged ? 1 : 0;
   plan->dtype = dtype;
   plan->policy = used_policy;
+  plan->ctas_per_unit = per;
+  plan->reserved = 0;
   plan->hist_len = hist_len;
-  plan->units = q_tiles * n_kv_heads * S;
+  plan->units = q_units * n_kv_heads * S;
   plan->scale = scale > 0.0f ? scale : (float)(1.0 / sqrt((double)head_dim));
   plan->est_us = (float)(simulate(num_sms, q_tiles, chunk_rows, G, n_kv_heads, hist_len, S,
                                   head_dim) +

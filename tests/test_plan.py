@@ -62,14 +62,18 @@ def P(**kw):
 
 def test_plan_fields(lib):
     p = P(splits=4)
-    assert p.group == 6 and p.q_tiles == 24 and p.splits == 4 and p.units == 24 * 4 * 4
+    # head dim 256 runs on CTA pairs: a unit is two consecutive Q tiles
+    assert p.group == 6 and p.q_tiles == 24 and p.splits == 4 and p.ctas_per_unit == 2
+    assert p.units == 12 * 4 * 4
     assert p.ws_bytes == 4 * 512 * 24 * 257 * 4
     assert abs(p.scale - 1 / 16) < 1e-7 and p.paged == 1 and p.policy == -1
 
 
 def test_plan_single_split_has_no_workspace(lib):
     p = P(splits=1)
-    assert p.ws_bytes == 0 and p.units == 96
+    assert p.ws_bytes == 0 and p.units == 48
+    q = P(splits=1, head_dim=128)
+    assert q.ctas_per_unit == 1 and q.units == 4 * q.q_tiles
 
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
@@ -89,7 +93,7 @@ def test_plan_workloads(lib, name):
 def test_makespan_policy_fills_the_gpu_at_long_history(lib):
     # 128 rows at 131072 history: 24 (tile, head) units alone would leave 124 SMs idle
     p = P(chunk_rows=128, hist_len=131072)
-    assert p.units >= 120
+    assert p.units * p.ctas_per_unit >= 120
     # an empty-history full chunk already fills the GPU: no split
     q = P(chunk_rows=2048, hist_len=0, n_q_heads=16, n_kv_heads=2, page_size=16, dtype="f16")
     assert q.splits == 1
