@@ -339,7 +339,15 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive(x.arrive_pfull + 8u * sbuf);
+      PA_TRACE_ONLY(if (threadIdx.x == 0) tlog(5, tln, 16, j);)
+      // P lives in tensor memory: a CTA-scope release orders it (see mbar_arrive_remote_tc);
+      // a tile whose V rows this thread zeroed in shared memory takes the cluster-scope one.
+      if (lane == 0) {
+        if (x.remote_arrive && !(PAGED && key0 + kTileKeys > a.total_keys))
+          mbar_arrive_remote_tc(x.arrive_pfull + 8u * sbuf);
+        else
+          arrive(x.arrive_pfull + 8u * sbuf);
+      }
       PA_TRACE_ONLY(tr[1] += clock64() - tc; if (threadIdx.x == 0) tlog(5, tln, 9, j);)
     }
 

@@ -9,10 +9,13 @@
 //   O += P V:   A = the two P tiles (each in its own tensor memory), B = V split by D (rank r
 //               holds dims 128r..128r+127 of all 128 keys).
 // Each CTA therefore loads half of every K/V tile: half the L2 traffic per FLOP of the
-// single-CTA kernel, and twice the time its shared-memory ring covers. Rank 1 tells rank 0
-// when its half of a slot has landed and when its Q and P are ready (remote mbarrier
-// arrivals); rank 0's MMA completions reach both CTAs (multicast commits). TMA loads always
-// fill the issuing CTA's own shared memory and signal its own barriers.
+// single-CTA kernel, and twice the time its shared-memory ring covers. Each CTA's copies fill
+// its own shared memory, and both halves of a slot complete on rank 0's barrier (the pair form
+// of the tensor copy), so rank 0 sees a slot as one unit. Rank 1 tells rank 0 when its Q and P
+// are ready (remote mbarrier arrivals); rank 0's MMA completions reach both CTAs (multicast
+// commits). One exception: the V rows of the sequence's last, partly filled tile complete on
+// the issuing CTA's own barrier, because its softmax warps zero the rows past the end before
+// the PV product reads them.
 
 struct PairCfg {
   static constexpr int NP = 4;        // 64-wide panels of a 256-wide row
@@ -20,11 +23,11 @@ struct PairCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NP * kPanel;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * kPanel;
-  // full[10], empty[10], peer_full[10] (rank 0: rank 1's half landed), q_full, s_full[2],
-  // p_full[2], pv_done[2], mma_done, teardown
-  static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_PEER = 2 * NSLOT, B_QFULL = 3 * NSLOT,
-                       B_SFULL = 3 * NSLOT + 1, B_PFULL = 3 * NSLOT + 3, B_PVDONE = 3 * NSLOT + 5,
-                       B_MMADONE = 3 * NSLOT + 7, B_TEAR = 3 * NSLOT + 8, N_BARS = 3 * NSLOT + 9;
+  // full[10] (rank 0: both halves landed), empty[10], q_full, s_full[2], p_full[2],
+  // pv_done[2], mma_done, teardown
+  static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_QFULL = 2 * NSLOT,
+                       B_SFULL = 2 * NSLOT + 1, B_PFULL = 2 * NSLOT + 3, B_PVDONE = 2 * NSLOT + 5,
+                       B_MMADONE = 2 * NSLOT + 7, B_TEAR = 2 * NSLOT + 8, N_BARS = 2 * NSLOT + 9;
   static constexpr int MISC_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int SMEM = MISC_OFF + 16;
   static constexpr int LAUNCH_SMEM = SMEM + 1024;
@@ -84,12 +87,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 4);
   const uint32_t leader_bar0 = mapa_shared(sb + C::BAR_OFF, 0);  // rank 0's barriers
   auto leader_bar = [&](int i) -> uint32_t { return leader_bar0 + 8u * (uint32_t)i; };
+  // The sequence's last KV tile, partly past the end (paged pools only: there the rows after
+  // the last key hold another sequence's data or nothing), is the unit's last tile; its V
+  // fills are the unit's last two (4n-2, 4n-1).
+  const bool has_tail = PAGED && (kt0 + n) * kTileKeys > a.total_keys;
+  auto tail_fill = [&](uint32_t q) -> bool { return has_tail && q + 2u >= 4u * (uint32_t)n; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(bar(C::B_FULL + i), 1);
       mbar_init(bar(C::B_EMPTY + i), 1);
-      mbar_init(bar(C::B_PEER + i), 1);
     }
     mbar_init(bar(C::B_QFULL), 8);   // 4 warps here + 4 warps of rank 1
     mbar_init(bar(C::B_SFULL + 0), 1);
@@ -157,12 +164,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.tmo = tmo;
     // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
     // is NaN inside the MMA, so this CTA's half of those V rows is zeroed before PV.
+    // Those fills complete on this CTA's own barrier: on rank 1 that barrier sees no other
+    // phase, so its parity is 0.
     auto v_tail = [&](int j, int r) -> bool {
       const uint32_t seq0 = v_item(j, n) * 2;
       bool okv = true;
       for (int k = 0; k < 2 && okv; ++k)
-        okv = warp_wait(bar(C::B_FULL + (seq0 + k) % NSLOT), ((seq0 + k) / NSLOT) & 1, abort_flag,
-                        tmo);
+        okv = warp_wait(bar(C::B_FULL + (seq0 + k) % NSLOT),
+                        rank == 0 ? ((seq0 + k) / NSLOT) & 1 : 0u, abort_flag, tmo);
       if (!okv || r < 0) return okv;
       for (int pl = 0; pl < 2; ++pl) {
         const uint32_t off = v_offset_pair((uint32_t)r, pl, a.v_shift);
@@ -209,14 +218,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t base = __shfl_sync(0xffffffffu, rows, pg & 31);
       return base == a.oob_row ? a.oob_row : base + (kk & (prow - 1));
     };
+    // Rank 0 expects both halves of a slot on its barrier; rank 1 arms its own barrier only for
+    // the tail fills.
     auto acquire = [&](uint32_t q) -> bool {
       const uint32_t slot = q % NSLOT;
+      PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 15, q);)
       bool r_ok = q < (uint32_t)NSLOT ||
                   warp_wait(bar(C::B_EMPTY + slot), ((q / NSLOT) - 1) & 1, abort_flag, tmo);
-      if (r_ok && lane == 0) mbar_arrive_expect_tx(bar(C::B_FULL + slot), kPanel);
+      if (r_ok && lane == 0) {
+        const bool tail = tail_fill(q);
+        if (rank == 0) mbar_arrive_expect_tx(bar(C::B_FULL + slot), tail ? kPanel : 2 * kPanel);
+        else if (tail) mbar_arrive_expect_tx(bar(C::B_FULL + slot), kPanel);
+      }
       __syncwarp();
       return r_ok;
     };
+    auto own_barrier = [&](uint32_t q) -> bool { return rank == 0 || tail_fill(q); };
     int32_t row_prev = a.oob_row, row_cur = fetch(0), row_next = fetch(1);
     uint32_t issued_end = 0;
     for (int j = 0; j <= n && ok; ++j) {
@@ -229,9 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((int)(q % kIssuers) != w) continue;
           if (!(ok = acquire(q))) break;
           const uint32_t slot = q % NSLOT;
-          if (l < 2 * k_per_panel)
-            tma_load_3d(slot_addr(slot) + pl * (kPanel / 2) + sub * k_rows * 128, &tm_k,
-                        bar(C::B_FULL + slot), (2 * k + pl) * 64, g, row);
+          if (l < 2 * k_per_panel) {
+            const uint32_t dst = slot_addr(slot) + pl * (kPanel / 2) + sub * k_rows * 128;
+            if (own_barrier(q))
+              tma_load_3d(dst, &tm_k, bar(C::B_FULL + slot), (2 * k + pl) * 64, g, row);
+            else
+              tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + slot), (2 * k + pl) * 64, g,
+                               row);
+          }
           issued_end = q + 1;
           PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 1, q);)
         }
@@ -244,9 +266,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((int)(q % kIssuers) != w) continue;
           if (!(ok = acquire(q))) break;
           const uint32_t slot = q % NSLOT;
-          if (lane < v_per_slot)
-            tma_load_4d(slot_addr(slot) + lane * (v_rows * 256), &tm_v, bar(C::B_FULL + slot), 0,
-                        row, 2 * (int)rank, g);
+          if (lane < v_per_slot) {
+            const uint32_t dst = slot_addr(slot) + lane * (v_rows * 256);
+            if (own_barrier(q))
+              tma_load_4d(dst, &tm_v, bar(C::B_FULL + slot), 0, row, 2 * (int)rank, g);
+            else
+              tma_load_4d_pair(dst, &tm_v, leader_bar(C::B_FULL + slot), 0, row, 2 * (int)rank,
+                               g);
+          }
           issued_end = q + 1;
           PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 2, q);)
         }
@@ -255,20 +282,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       row_cur = row_next;
       row_next = fetch(j + 2);
     }
-    // Wait for this warp's copies among the last NSLOT fills (see the single-CTA kernel).
+    // Wait for this warp's copies among the last NSLOT fills (see the single-CTA kernel). On
+    // rank 0 the barrier covers both halves, so rank 1's copies have landed as well; rank 1
+    // drains only the tail fills on its own barrier, and it stays resident until rank 0 has
+    // finished (teardown handshake below).
     const uint32_t all_fills = 4u * n;
     for (uint32_t q = all_fills > (uint32_t)NSLOT ? all_fills - NSLOT : 0; q < issued_end; ++q)
-      if ((int)(q % kIssuers) == w)
-        drain_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo);
+      if ((int)(q % kIssuers) == w && own_barrier(q))
+        drain_wait(bar(C::B_FULL + q % NSLOT), rank == 0 ? (q / NSLOT) & 1 : 0u, abort_flag,
+                   tmo);
     __syncwarp();
   } else if (rank == 0) {
     // ============================================================ MMA issuer (rank 0, one lane)
-    PA_TRACE_ONLY(if (lane == 1) {
-      for (uint32_t q = 0; q < 4u * n; ++q) {
-        if (!thread_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo)) break;
-        tlog(4, tln, 10, q);
-      }
-    })
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_f16(256, kTileKeys, BF16, false);
       constexpr uint32_t idesc_pv = umma_idesc_f16(256, D, BF16, true);
@@ -279,10 +304,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t v_desc =
           smem_desc_sw128(sb + C::RING_OFF, (uint32_t)(1 << a.v_shift) * 128u, 1024);
       uint32_t slot = 0, round = 0;
-      // a slot is ready when both halves landed: this CTA's (local) and rank 1's (relayed)
+      PA_TRACE_ONLY(unsigned tln_w = 0;)
+      // a slot is ready when both halves landed (one barrier; for the tail fills rank 1's half
+      // is covered by its softmax warps' P-ready arrival, which waits for it)
       auto wait_slot = [&]() -> bool {
-        return thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo) &&
-               wait_cluster(bar(C::B_PEER + slot), round & 1);
+        PA_TRACE_ONLY(tlog(6, tln_w, 11, round * NSLOT + slot);)
+        return thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
       };
       auto advance = [&]() {
         if (++slot == (uint32_t)NSLOT) {
@@ -319,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (j >= 1) {
           const int i = j - 1;
+          PA_TRACE_ONLY(tlog(6, tln_w, 14, i);)
           ok = wait_cluster(bar(C::B_PFULL + (i & 1)), (i >> 1) & 1);
           PA_TRACE_ONLY(tlog(3, tln, 5, i);)
           const uint32_t vslot0 = slot;
@@ -353,18 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ============================================================ relay (rank 1, one lane)
-    // Tell rank 0 when this CTA's half of each slot has landed, in fill order.
-    if (lane == 0) {
-      const uint32_t all_fills = 4u * n;
-      for (uint32_t q = 0; q < all_fills; ++q) {
-        if (!thread_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo)) break;
-        PA_TRACE_ONLY(tlog(4, tln, 10, q);)
-        mbar_arrive_remote(leader_bar(C::B_PEER + q % NSLOT));
-      }
-      // rank 0's last MMA has read this CTA's shared and tensor memory
-      drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
-    }
+    // ============================================================ rank 1, MMA warp
+    // rank 0's last MMA has read this CTA's shared and tensor memory
+    if (lane == 0) drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
     __syncwarp();
   }
 
