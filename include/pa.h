@@ -49,15 +49,24 @@ typedef enum {
 
 /* Split policies for pa_plan (how the history of a piece is partitioned). */
 typedef enum {
-  /* B200: the split count that minimises the simulated makespan of the launch on
-   * num_sms SMs (units are dispatched longest first), plus the combine's HBM cost. */
+  /* B200: the schedule that minimises the simulated makespan of the launch on num_sms SMs
+   * (items are dispatched in order to the first free SM), plus the combine's HBM cost: a
+   * uniform split count (units longest first), or the balanced schedule when it is faster. */
   PA_POLICY_MAKESPAN = 0,
   /* The rule of splash PR #33 ("What changed"): min(256, max(32, 32*cores/kv_heads)) /
    * tiles, clamped to 1..32, with cores = num_sms and tiles = Q tiles per KV head. */
   PA_POLICY_CORES = 1,
   /* The earlier rule quoted in splash PR #33: clamp(32 / tiles, 1, 32), with tiles taken as
    * the threadgroups over all KV heads (the reading under which every listed piece got 1). */
-  PA_POLICY_LEGACY = 2
+  PA_POLICY_LEGACY = 2,
+  /* B200: cut the history of some row blocks at arbitrary KV tiles so that every SM (or SM
+   * pair) gets the same number of KV tiles: the row blocks' tiles are laid end to end and cut
+   * where each worker's equal share ends (McNaughton's wrap-around rule), no piece shorter
+   * than a few tiles. Uncut row blocks write `out` directly; the parts of a cut one are merged
+   * by pa_combine. Falls back to the makespan policy's uniform splits only when the
+   * schedule would not fit the kernel's tables (512 items, 256 cut row blocks, 32 parts);
+   * the plan's `policy` field says which was used. */
+  PA_POLICY_BALANCED = 3
 } pa_policy;
 
 /* Rows of the packed (token, head) Q tile, and keys per KV tile, of the kernel. */
@@ -75,6 +84,12 @@ typedef enum {
  * [s*n/S, (s+1)*n/S) of the n = ceil((H + t_last + 1) / PA_TILE_KEYS) tiles it sees. With
  * ctas_per_unit = 2 a unit is a pair of consecutive Q tiles (2t, 2t+1) on a CTA pair, and t_last
  * is that of the pair's last tile.
+ *
+ * Plans with policy == PA_POLICY_BALANCED use work items instead of uniform splits. A row
+ * block is (unit of ctas_per_unit Q tiles, KV head), numbered rb = (q_units-1-u)*Hkv + g with
+ * q_units = ceil(q_tiles / ctas_per_unit) (last unit first); an item is a run [kt0, kt1) of
+ * the KV tiles its unit sees; `units` counts the items and `splits` is the largest number of
+ * items of one row block. pa_schedule_items lists them.
  */
 typedef struct {
   int32_t num_sms;        /* SMs the plan was made for */
@@ -85,17 +100,21 @@ typedef struct {
   int32_t group;          /* G = Hq / Hkv */
   int32_t chunk_rows;     /* R: query rows of the piece (>= 1) */
   int32_t q_tiles;        /* ceil(R * G / PA_TILE_ROWS) per KV head */
-  int32_t splits;         /* S: 1..PA_MAX_SPLITS */
+  int32_t splits;         /* S: 1..PA_MAX_SPLITS (balanced: most items of one row block) */
   int32_t paged;          /* 1: k/v are page pools read through page_table; 0: contiguous */
   int32_t dtype;          /* pa_dtype of q, k, v */
-  int32_t policy;         /* pa_policy used (or -1 when splits was overridden) */
+  int32_t policy;         /* pa_policy used (or -1 when splits was overridden); balanced
+                           * plans read PA_POLICY_BALANCED whichever policy chose them */
   int32_t ctas_per_unit;  /* 2: head_dim 256 runs on CTA pairs (two Q tiles per unit); else 1 */
   int32_t reserved;
   int64_t hist_len;       /* H: keys in the cache before the piece */
-  int64_t units;          /* Hkv * ceil(q_tiles / ctas_per_unit) * S units (CTAs or pairs) */
+  int64_t units;          /* Hkv * ceil(q_tiles / ctas_per_unit) * S units (CTAs or pairs);
+                           * balanced: the number of items */
   float scale;            /* softmax scale actually used */
   float est_us;           /* the planner's time estimate for prefill + combine (microseconds) */
-  uint64_t ws_bytes;      /* bytes of lse_ws needed: S*R*Hq*(D+1)*4 if S > 1, else 0 */
+  uint64_t ws_bytes;      /* bytes of lse_ws needed: S*R*Hq*(D+1)*4 if S > 1, else 0;
+                           * balanced: slots * ctas_per_unit*128 * (D+1) * 4, one slot per
+                           * item of a cut row block */
 } pa_plan_t;
 
 /*
@@ -116,6 +135,15 @@ int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_s
             int policy, int paged, pa_plan_t* plan);
 
 /*
+ * pa_schedule_items — the work items of a balanced plan, in launch order: for item i,
+ * items[4i..4i+3] = (rb, kt0, kt1, slot), slot = -1 for an uncut row block (written to out)
+ * or the workspace slot of its partial. Writes at most `cap` items (items may be NULL).
+ * Returns the number of items, 0 for a plan that is not balanced, or PA_ERR_INVALID_ARG when
+ * the plan does not match its own schedule. Pure host code.
+ */
+int pa_schedule_items(const pa_plan_t* plan, int32_t* items, int cap);
+
+/*
  * pa_prefill — split-KV prefill attention of one piece, enqueued on `stream`.
  *   q            device, [R][Hq][D] of dtype, contiguous, 16-byte aligned.
  *   k_pool,v_pool device, paged: [num_pages][PS][Hkv][D]; contiguous: [H+R][Hkv][D]; dtype,
@@ -126,11 +154,15 @@ int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_s
  *                and raises PA_ERR_PAGE_INDEX in pa_device_error.
  *   num_pages    pages in each pool (paged only).
  *   hist_len, chunk_rows: must equal the plan's.
- *   out          device fp32 [R][Hq][D]. Written when plan->splits == 1.
+ *   out          device fp32 [R][Hq][D]. Written when plan->splits == 1; balanced plans
+ *                write the rows of uncut row blocks here.
  *   lse_ws       device fp32 workspace of ws_bytes >= plan->ws_bytes (used when S > 1):
  *                partial outputs O_s [S][R][Hq][D] (each normalised over its split), then
  *                base-2 log-sum-exp of the scaled scores lse_s [S][R][Hq] (-inf: no key).
- * When S > 1, call pa_combine afterwards on the same stream to produce `out`.
+ *                Balanced plans: O [slots][rows][D] then lse [slots][rows], rows =
+ *                ctas_per_unit*128 packed rows of the item's row block.
+ * When S > 1 (or the plan is balanced with a cut row block), call pa_combine afterwards on
+ * the same stream to produce `out`.
  * Returns PA_OK or an error status; launch errors are PA_ERR_CUDA. Device-side conditions
  * (bad page entry, wait timeout) are reported by pa_device_error.
  */
@@ -141,7 +173,8 @@ int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_pool, const v
 /*
  * pa_combine — log-sum-exp merge of the S split partials in lse_ws into out (fp32
  * [R][Hq][D]): out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s.
- * No-op returning PA_OK when plan->splits == 1. Source: splash PR #33, the prefill
+ * No-op returning PA_OK when plan->splits == 1. For balanced plans it merges the parts of
+ * each cut row block into that block's rows of out. Source: splash PR #33, the prefill
  * attention "reduce" that merges the split partials (decode-profile tables).
  */
 int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes, float* out,

@@ -15,13 +15,14 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(PKG, "libpa.so")
 
 PA_F16, PA_BF16 = 0, 1
-POLICIES = {"makespan": 0, "cores": 1, "legacy": 2}
+POLICIES = {"makespan": 0, "cores": 1, "legacy": 2, "balanced": 3}
+PA_POLICY_BALANCED = 3
 STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
           -4: "PA_ERR_CUDA", -5: "PA_ERR_TIMEOUT", -6: "PA_ERR_PAGE_INDEX"}
 EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_device_error",
             "pa_set_wait_timeout_ns",
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
-            "pa_legacy_policy_splits")
+            "pa_legacy_policy_splits", "pa_schedule_items")
 
 
 class PaError(RuntimeError):
@@ -83,6 +84,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_cores_policy_splits.restype = i32
     lib.pa_legacy_policy_splits.argtypes = [i32, i32]
     lib.pa_legacy_policy_splits.restype = i32
+    lib.pa_schedule_items.argtypes = [ctypes.POINTER(Plan), ctypes.POINTER(ctypes.c_int32), i32]
+    lib.pa_schedule_items.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -115,6 +118,18 @@ def plan(n_q_heads: int, n_kv_heads: int, head_dim: int, page_size: int, chunk_r
                                 1 if paged else 0, ctypes.byref(p))
     _check(st, "pa_plan")
     return p
+
+
+def schedule_items(p: Plan):
+    """pa_schedule_items: the work items of a balanced plan as an int32 array [n, 4] of
+    (row block, kt0, kt1, workspace slot or -1); empty for other plans."""
+    import numpy as np
+    lib = load_library()
+    n = lib.pa_schedule_items(ctypes.byref(p), None, 0)
+    _check(0 if n >= 0 else n, "pa_schedule_items")
+    buf = (ctypes.c_int32 * max(4 * n, 1))()
+    lib.pa_schedule_items(ctypes.byref(p), buf, n)
+    return np.frombuffer(buf, dtype=np.int32)[:4 * n].reshape(n, 4).copy()
 
 
 def _stream_ptr(stream):
@@ -169,10 +184,10 @@ def prefill(p: Plan, q, k_pool, v_pool, page_table, out, ws=None, stream=None):
             raise ValueError("contiguous k/v must be [H+R, Hkv, D]")
         num_pages, tab = 0, None
     out_ptr, ws_ptr, ws_bytes = None, None, 0
-    if p.splits == 1:
+    if p.splits == 1 or p.policy == PA_POLICY_BALANCED:
         _require_cuda(out, "out", torch.float32, (R, Hq, D))
         out_ptr = out.data_ptr()
-    else:
+    if p.ws_bytes > 0:
         _require_cuda(ws, "ws", torch.float32)
         ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * 4
     st = load_library().pa_prefill(ctypes.byref(p), q.data_ptr(), k_pool.data_ptr(),
@@ -182,9 +197,9 @@ def prefill(p: Plan, q, k_pool, v_pool, page_table, out, ws=None, stream=None):
 
 
 def combine(p: Plan, ws, out, stream=None):
-    """pa_combine: merge split partials into out (no-op when splits == 1)."""
+    """pa_combine: merge split partials into out (no-op when there are none)."""
     import torch
-    if p.splits == 1:
+    if p.ws_bytes == 0:
         return
     _require_cuda(ws, "ws", torch.float32)
     _require_cuda(out, "out", torch.float32, (p.chunk_rows, p.n_q_heads, p.head_dim))
@@ -199,7 +214,7 @@ def prefill_combine(p: Plan, q, k_pool, v_pool, page_table, out=None, ws=None, s
     if out is None:
         out = torch.empty((p.chunk_rows, p.n_q_heads, p.head_dim), dtype=torch.float32,
                           device=q.device)
-    if p.splits > 1 and ws is None:
+    if p.ws_bytes > 0 and ws is None:
         ws = workspace(p, q.device)
     prefill(p, q, k_pool, v_pool, page_table, out, ws, stream)
     combine(p, ws, out, stream)

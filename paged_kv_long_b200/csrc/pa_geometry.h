@@ -64,4 +64,26 @@ PA_HD void unit_coords(int64_t u, int64_t q_tiles, int Hkv, int S, int64_t* qt, 
   *s = (int)(rem % S);
 }
 
+// ---- balanced schedule (plans made with the balanced policy)
+//
+// A row block is (unit of `per` consecutive Q tiles, KV head): rb = (q_units-1-qu)*Hkv + g,
+// longest first. A work item is a contiguous run [kt0, kt1) of a row block's visible KV
+// tiles; `slot` is the workspace slot of its partial, or -1 when the item is the whole row
+// block and writes the final output.
+struct PaItem {
+  int32_t rb, kt0, kt1, slot;
+};
+// Row block that was cut into nparts items, whose partials sit in workspace slots
+// [first_slot, first_slot + nparts).
+struct PaSplitBlock {
+  int32_t rb, first_slot, nparts, pad;
+};
+constexpr int kMaxItems = 512;
+constexpr int kMaxSplitBlocks = 256;
+
+PA_HD void rb_coords(int32_t rb, int64_t q_units, int Hkv, int64_t* qu, int* g) {
+  *qu = q_units - 1 - rb / Hkv;
+  *g = rb % Hkv;
+}
+
 }  // namespace pa

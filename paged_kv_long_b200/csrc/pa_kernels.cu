@@ -32,6 +32,7 @@
 
 #include "pa.h"
 #include "pa_geometry.h"
+#include "pa_schedule.h"
 #include "sm100.cuh"
 
 namespace pa {
@@ -71,7 +72,17 @@ struct PrefillArgs {
   int32_t oob_row;       // a key-row coordinate past the pool: the TMA fills zeros there
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
+  int32_t balanced;        // 1: CTA (pair) b runs work item b of the item table
+  int32_t rows_per_block;  // packed rows of a row block (balanced workspace slots)
 };
+
+// The work items of a balanced plan, passed by value (kernel parameter space): no device
+// allocation, and a CUDA graph that captures the launch keeps its own copy.
+struct ItemTable {
+  PaItem item[kMaxItems];
+};
+// SoftmaxCtx::slot value of the uniform-split schedule (destination from the split index).
+constexpr int kSlotUniform = -2;
 
 // Shared-memory layout. The ring holds 16 KB slots, filled and consumed in the order K0, K1,
 // V0, K2, V1, ..., V_{n-1}; every K or V tile takes NP consecutive slots (mod NSLOT). A K
@@ -108,6 +119,20 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
   return ((k >> v_shift) << (v_shift + PANEL_LOG)) + ((p << v_shift) << 7) +
          ((k & ((1u << v_shift) - 1u)) << 7);
 }
+
+#ifdef PA_UNIT_TIMING
+// Instrumented builds only: per CTA (blockIdx < 8192) the global timer at entry and at exit,
+// its key-tile count and its SM (see pa_unit_timing).
+__device__ unsigned long long g_pa_units[4 * 8192];
+__device__ __forceinline__ uint32_t smid_u32() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
+#define PA_UNIT_ONLY(...) __VA_ARGS__
+#else
+#define PA_UNIT_ONLY(...)
+#endif
 
 #ifdef PA_TRACE
 // Instrumented builds only: cycle counters summed over all CTAs (see pa_trace_read), and an
@@ -189,6 +214,9 @@ struct SoftmaxCtx {
   int g, s;
   int64_t kt0;
   int n;
+  int slot;       // workspace slot of a balanced item's partial, -1: final output,
+                  // kSlotUniform: uniform splits (out when S == 1, else split s's partial)
+  int row0;       // first packed row of this CTA inside its row block (balanced slots)
   volatile int* abort_flag;
   uint64_t tmo;
 };
@@ -358,8 +386,12 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
     if (ok) {
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      float* dst = (a.splits == 1) ? a.out + (tok * a.Hq + head) * (int64_t)D
-                                   : a.ws_o + (((int64_t)s * a.R + tok) * a.Hq + head) * D;
+      int64_t ws_row = -1;  // workspace row of a partial; -1: the final output
+      if (x.slot >= 0)
+        ws_row = (int64_t)x.slot * a.rows_per_block + x.row0 + r;
+      else if (x.slot == kSlotUniform && a.splits > 1)
+        ws_row = ((int64_t)s * a.R + tok) * a.Hq + head;
+      float* dst = ws_row < 0 ? a.out + (tok * a.Hq + head) * (int64_t)D : a.ws_o + ws_row * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
@@ -373,9 +405,7 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
                                 o[4 * i + 3] * inv_l);
         }
       }
-      if (valid && a.splits > 1)
-        a.ws_lse[((int64_t)s * a.R + tok) * a.Hq + head] =
-            l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+      if (valid && ws_row >= 0) a.ws_lse[ws_row] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
     }
     PA_TRACE_ONLY(tr[2] += clock64() - te;
                   if (lane == 0) {
@@ -393,7 +423,7 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
 template <int D, bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const PrefillArgs a) {
+                   const PrefillArgs a, const __grid_constant__ ItemTable items) {
   using C = Cfg<D>;
   constexpr int NP = C::NP, NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
@@ -402,12 +432,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  int64_t qt;
-  int g, s;
-  unit_coords(blockIdx.x, a.q_tiles, a.Hkv, a.splits, &qt, &g, &s);
-  const int64_t n_kt_all = tile_kv_tiles(qt, a.R, a.G, a.hist_len);
-  int64_t kt0, kt1;
-  split_range(n_kt_all, s, a.splits, &kt0, &kt1);
+  int64_t qt, kt0, kt1;
+  int g, s, slot = kSlotUniform;
+  if (a.balanced) {
+    const PaItem it = items.item[blockIdx.x];
+    rb_coords(it.rb, a.q_tiles, a.Hkv, &qt, &g);
+    s = 0;
+    kt0 = it.kt0;
+    kt1 = it.kt1;
+    slot = it.slot;
+  } else {
+    unit_coords(blockIdx.x, a.q_tiles, a.Hkv, a.splits, &qt, &g, &s);
+    split_range(tile_kv_tiles(qt, a.R, a.G, a.hist_len), s, a.splits, &kt0, &kt1);
+  }
   const int n = (int)(kt1 - kt0);
 
   if (n == 0) {  // a split past this tile's keys (only when S > KV tiles): empty partial
@@ -478,6 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.s = s;
     sc.kt0 = kt0;
     sc.n = n;
+    sc.slot = slot;
+    sc.row0 = 0;
     sc.abort_flag = abort_flag;
     sc.tmo = tmo;
     // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
@@ -720,6 +759,57 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   }
 }
 
+// Balanced plans: one warp per packed row of a cut row block merges that row's parts (workspace
+// slots first_slot .. first_slot + nparts - 1, at most 32) into out, with the same weighting.
+struct SplitTable {
+  PaSplitBlock blk[kMaxSplitBlocks];
+};
+
+__global__ void __launch_bounds__(256) combine_blocks_kernel(
+    const float* __restrict__ ws_o, const float* __restrict__ ws_lse, float* __restrict__ out,
+    const __grid_constant__ SplitTable t, int n_blocks, int rows_per_block, int64_t q_units,
+    int Hkv, int G, int R, int Hq, int D) {
+  const int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (w >= (int64_t)n_blocks * rows_per_block) return;
+  const int lane = threadIdx.x & 31;
+  const PaSplitBlock b = t.blk[w / rows_per_block];
+  const int lr = (int)(w % rows_per_block);
+  int64_t qu;
+  int g;
+  rb_coords(b.rb, q_units, Hkv, &qu, &g);
+  const int64_t grow = qu * rows_per_block + lr;
+  const int64_t tok = grow / G;
+  if (tok >= R) return;
+  const int head = g * G + (int)(grow % G);
+  const int64_t row0 = (int64_t)b.first_slot * rows_per_block + lr;  // part p: row0 + p * rpb
+  const float lse = lane < b.nparts ? ws_lse[row0 + (int64_t)lane * rows_per_block] : -INFINITY;
+  float M = lse;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float wt = (lse == -INFINITY) ? 0.f : exp2f(lse - M);
+  float W = wt;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  float* dst = out + (tok * Hq + head) * (int64_t)D;
+  for (int d0 = lane * 4; d0 < D; d0 += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < b.nparts; ++sp) {
+      const float ws = __shfl_sync(0xffffffffu, wt, sp);
+      if (ws != 0.f) {
+        const float4 o =
+            *reinterpret_cast<const float4*>(ws_o + (row0 + (int64_t)sp * rows_per_block) * D + d0);
+        acc.x = fmaf(ws, o.x, acc.x);
+        acc.y = fmaf(ws, o.y, acc.y);
+        acc.z = fmaf(ws, o.z, acc.z);
+        acc.w = fmaf(ws, o.w, acc.w);
+      }
+    }
+    *reinterpret_cast<float4*>(dst + d0) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+}
+
 // ---------------------------------------------------------------- timeout self-test
 __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
   __shared__ __align__(8) uint64_t never;
@@ -790,7 +880,7 @@ bool make_v_map(CUtensorMap* map, const void* base, bool bf16, int D, int Hkv, i
 
 template <int D, bool PAGED, bool BF16>
 cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
-                           const CUtensorMap& tv, const PrefillArgs& a) {
+                           const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
   auto kern = prefill_kernel<D, PAGED, BF16>;
   static std::atomic<uint64_t> configured{0};  // one bit per device ordinal
   int dev = 0;
@@ -803,13 +893,13 @@ cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  kern<<<(unsigned)grid, kThreads, Cfg<D>::LAUNCH_SMEM, st>>>(tk, tv, a);
+  kern<<<(unsigned)grid, kThreads, Cfg<D>::LAUNCH_SMEM, st>>>(tk, tv, a, it);
   return cudaGetLastError();
 }
 
 template <bool PAGED, bool BF16>
 cudaError_t launch_pair(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
-                        const CUtensorMap& tv, const PrefillArgs& a) {
+                        const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
   auto kern = prefill_pair_kernel<PAGED, BF16>;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -834,19 +924,19 @@ cudaError_t launch_pair(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a);
+  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a, it);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(bool paged, bool bf16, int64_t grid, cudaStream_t st, const CUtensorMap& tk,
-                     const CUtensorMap& tv, const PrefillArgs& a) {
+                     const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
   if (paged)
-    return bf16 ? launch_prefill<D, true, true>(grid, st, tk, tv, a)
-                : launch_prefill<D, true, false>(grid, st, tk, tv, a);
-  return bf16 ? launch_prefill<D, false, true>(grid, st, tk, tv, a)
-              : launch_prefill<D, false, false>(grid, st, tk, tv, a);
+    return bf16 ? launch_prefill<D, true, true>(grid, st, tk, tv, a, it)
+                : launch_prefill<D, true, false>(grid, st, tk, tv, a, it);
+  return bf16 ? launch_prefill<D, false, true>(grid, st, tk, tv, a, it)
+              : launch_prefill<D, false, false>(grid, st, tk, tv, a, it);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -870,9 +960,15 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
     return PA_ERR_INVALID_ARG;
   const int64_t total_keys = hist_len + chunk_rows;
   const int S = plan->splits;
-  if (S == 1) {
+  const bool balanced = plan->policy == PA_POLICY_BALANCED;
+  Schedule sch;
+  if (balanced && (!build_balanced(*plan, &sch) || (int64_t)sch.items.size() != plan->units))
+    return PA_ERR_INVALID_ARG;
+  const bool partials = balanced ? sch.n_slots > 0 : S > 1;
+  if (balanced || S == 1) {
     if (!out || !aligned16(out)) return PA_ERR_INVALID_ARG;
-  } else {
+  }
+  if (partials) {
     if (!lse_ws || !aligned16(lse_ws) || ws_bytes < plan->ws_bytes) return PA_ERR_WORKSPACE;
   }
   const bool paged = plan->paged != 0;
@@ -886,7 +982,8 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   if (per != (D == 256 ? 2 : 1)) return PA_ERR_INVALID_ARG;
   const int64_t q_units = ((int64_t)plan->q_tiles + per - 1) / per;
   const int64_t grid = plan->units * per;  // CTAs
-  if (plan->units != q_units * plan->n_kv_heads * S || grid <= 0 || grid >= (int64_t(1) << 31))
+  const int64_t want_units = balanced ? (int64_t)sch.items.size() : q_units * plan->n_kv_heads * S;
+  if (plan->units != want_units || grid <= 0 || grid >= (int64_t(1) << 31))
     return PA_ERR_INVALID_ARG;
 
   CUtensorMap tk, tv;
@@ -905,8 +1002,10 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.q = static_cast<const uint16_t*>(q);
   a.page_table = page_table;
   a.out = out;
-  a.ws_o = S > 1 ? lse_ws : nullptr;
-  a.ws_lse = S > 1 ? lse_ws + (int64_t)S * chunk_rows * plan->n_q_heads * D : nullptr;
+  a.ws_o = partials ? lse_ws : nullptr;
+  a.ws_lse = !partials ? nullptr
+             : balanced ? lse_ws + (int64_t)sch.n_slots * sch.rows_per_block * D
+                        : lse_ws + (int64_t)S * chunk_rows * plan->n_q_heads * D;
   a.hist_len = hist_len;
   a.table_len = paged ? (total_keys + PS - 1) / PS : 0;
   a.total_keys = total_keys;
@@ -926,17 +1025,24 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.oob_row = (int32_t)rows;
   a.scale_log2 = plan->scale * 1.4426950408889634f;
   a.timeout_ns = g_timeout_ns.load();
+  a.balanced = balanced ? 1 : 0;
+  a.rows_per_block = per * kTileRows;
+  // Kernel parameter of 8 KB, copied into the launch: kept off the stack of callers with small
+  // stacks, one per thread (the launch has taken its copy when this function returns).
+  thread_local ItemTable table;
+  ItemTable* tab = &table;
+  for (size_t i = 0; i < sch.items.size(); ++i) tab->item[i] = sch.items[i];
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   switch (D) {
-    case 64: e = launch_d<64>(paged, bf16, grid, st, tk, tv, a); break;
-    case 128: e = launch_d<128>(paged, bf16, grid, st, tk, tv, a); break;
+    case 64: e = launch_d<64>(paged, bf16, grid, st, tk, tv, a, *tab); break;
+    case 128: e = launch_d<128>(paged, bf16, grid, st, tk, tv, a, *tab); break;
     default:
-      e = paged ? (bf16 ? launch_pair<true, true>(grid, st, tk, tv, a)
-                        : launch_pair<true, false>(grid, st, tk, tv, a))
-                : (bf16 ? launch_pair<false, true>(grid, st, tk, tv, a)
-                        : launch_pair<false, false>(grid, st, tk, tv, a));
+      e = paged ? (bf16 ? launch_pair<true, true>(grid, st, tk, tv, a, *tab)
+                        : launch_pair<true, false>(grid, st, tk, tv, a, *tab))
+                : (bf16 ? launch_pair<false, true>(grid, st, tk, tv, a, *tab)
+                        : launch_pair<false, false>(grid, st, tk, tv, a, *tab));
       break;
   }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -946,6 +1052,27 @@ extern "C" int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t w
                           float* out, pa_stream_t stream) {
   if (!plan) return PA_ERR_INVALID_ARG;
   const int S = plan->splits;
+  if (plan->policy == PA_POLICY_BALANCED) {
+    Schedule sch;
+    if (!build_balanced(*plan, &sch) || (int64_t)sch.items.size() != plan->units)
+      return PA_ERR_INVALID_ARG;
+    if (sch.split.empty()) return PA_OK;
+    if (sch.max_parts > 32) return PA_ERR_INVALID_ARG;
+    if (!lse_ws || ws_bytes < plan->ws_bytes || !aligned16(lse_ws)) return PA_ERR_WORKSPACE;
+    if (!out || !aligned16(out)) return PA_ERR_INVALID_ARG;
+    thread_local SplitTable table;
+    for (size_t i = 0; i < sch.split.size(); ++i) table.blk[i] = sch.split[i];
+    const int D = plan->head_dim;
+    const int per = plan->ctas_per_unit;
+    const int64_t q_units = ((int64_t)plan->q_tiles + per - 1) / per;
+    const int64_t warps = (int64_t)sch.split.size() * sch.rows_per_block;
+    combine_blocks_kernel<<<(unsigned)((warps + 7) / 8), 256, 0,
+                            reinterpret_cast<cudaStream_t>(stream)>>>(
+        lse_ws, lse_ws + (int64_t)sch.n_slots * sch.rows_per_block * D, out, table,
+        (int)sch.split.size(), sch.rows_per_block, q_units, plan->n_kv_heads, plan->group,
+        plan->chunk_rows, plan->n_q_heads, D);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
   if (S == 1) return PA_OK;
   if (S < 1 || S > PA_MAX_SPLITS) return PA_ERR_INVALID_ARG;
   if (!lse_ws || ws_bytes < plan->ws_bytes || !aligned16(lse_ws)) return PA_ERR_WORKSPACE;
@@ -991,7 +1118,7 @@ extern "C" int pa_prefill_noalloc(const pa_plan_t* plan, const void* q, const vo
   if (!plan) return PA_ERR_INVALID_ARG;
   float* ws = nullptr;
   uint64_t ws_bytes = 0;
-  if (plan->splits > 1) {
+  if (plan->ws_bytes > 0) {
     if (plan->ws_bytes > PA_NOALLOC_WS_BYTES) return PA_ERR_WORKSPACE;
     const int st = noalloc_scratch(&ws);
     if (st != PA_OK) return st;
@@ -1017,6 +1144,19 @@ extern "C" int pa_device_error(int* flags, int reset) {
   if (v & kFlagTimeout) return PA_ERR_TIMEOUT;
   return PA_OK;
 }
+
+#ifdef PA_UNIT_TIMING
+extern "C" int pa_unit_timing(unsigned long long* out, int cap, int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  int n = cap < 4 * 8192 ? cap : 4 * 8192;
+  if (cudaMemcpyFromSymbol(out, g_pa_units, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
+  if (reset) {
+    static unsigned long long z[4 * 8192];
+    cudaMemcpyToSymbol(g_pa_units, z, sizeof z);
+  }
+  return n;
+}
+#endif
 
 #ifdef PA_TRACE
 extern "C" int pa_trace_log(unsigned long long* out, int cap, int reset) {

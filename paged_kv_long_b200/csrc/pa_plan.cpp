@@ -18,6 +18,7 @@
 
 #include "pa.h"
 #include "pa_geometry.h"
+#include "pa_schedule.h"
 
 namespace {
 
@@ -75,7 +76,132 @@ double combine_cost(int S, int64_t R, int Hq, int D) {
   return bytes * cm.combine_us_per_byte + cm.combine_fixed_us;
 }
 
+// Greedy dispatch of items, in order, to `slots` identical workers (what the hardware does
+// with a grid of CTAs that each hold a whole SM or SM pair).
+double simulate_items(const std::vector<pa::PaItem>& items, int slots, const CostModel& cm) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> q;
+  for (int i = 0; i < slots; ++i) q.push(0.0);
+  double makespan = 0.0;
+  for (const pa::PaItem& it : items) {
+    const double t = q.top() + (it.kt1 - it.kt0) * cm.tile_us + cm.unit_us;
+    q.pop();
+    q.push(t);
+    makespan = std::max(makespan, t);
+  }
+  return makespan;
+}
+
 }  // namespace
+
+namespace pa {
+
+// McNaughton's wrap-around rule over the row blocks' KV tiles: lay the row blocks end to end
+// (longest first), fill `slots` workers to an equal load in turn, and cut a row block where a
+// worker's share ends. Every worker then carries the same load and at most one cut per worker
+// boundary is made; no piece shorter than `m` tiles is cut off. Items are issued in the order of
+// their planned start, so the hardware's first-free-SM dispatch reproduces the plan.
+bool build_balanced(const pa_plan_t& p, Schedule* out) {
+  const CostModel cm(p.head_dim);
+  const int per = ctas_per_unit_for(p.head_dim);
+  const int slots = std::max(1, p.num_sms / per);
+  const int64_t q_units = ((int64_t)p.q_tiles + per - 1) / per;
+  const int Hkv = p.n_kv_heads;
+  const int64_t n_rb = q_units * Hkv;
+  if (n_rb > kMaxItems) return false;
+  std::vector<int64_t> len(n_rb);
+  double total = 0.0;
+  for (int64_t rb = 0; rb < n_rb; ++rb) {
+    int64_t qu;
+    int g;
+    rb_coords((int32_t)rb, q_units, Hkv, &qu, &g);
+    len[rb] = unit_kv_tiles(qu, per, p.q_tiles, p.chunk_rows, p.group, p.hist_len);
+    total += (double)len[rb];
+  }
+  const double c_item = cm.unit_us / cm.tile_us;  // fixed cost of an item, in tiles
+  struct Piece {
+    int32_t rb, kt0, kt1, worker;
+    double start;
+  };
+  std::vector<Piece> pieces;
+  // Wrap-around assignment for a given share per worker; returns the workers it needs.
+  auto assign = [&](double share, int64_t m, double over) -> int {
+    pieces.clear();
+    int k = 0;
+    double load = 0.0;
+    for (int64_t rb = 0; rb < n_rb; ++rb) {
+      int64_t o = 0, r = len[rb];
+      while (r > 0) {
+        const double room = share - load - c_item;
+        int64_t take;
+        if ((double)r <= room + over) {
+          take = r;  // the rest fits (a little over is fine)
+        } else if (load > 0.0 && room < (double)m) {
+          ++k;       // this worker is full
+          load = 0.0;
+          if (k > slots) return k + 1;  // cannot fit: stop early
+          continue;
+        } else {
+          // at least m tiles (a fresh worker always makes progress), and leave at least m
+          take = std::max<int64_t>((int64_t)room, m);
+          if (r - take < m) take = r;
+        }
+        pieces.push_back({(int32_t)rb, (int32_t)o, (int32_t)(o + take), k, load});
+        load += (double)take + c_item;
+        o += take;
+        r -= take;
+        if (r > 0) {
+          ++k;
+          load = 0.0;
+        }
+      }
+    }
+    return k + 1;
+  };
+  // The smallest share (from the even split of the tiles plus one item cost per row block and
+  // per cut) whose assignment fits the workers.
+  double share = (total + c_item * (double)(n_rb + slots - 1)) / slots;
+  const int64_t m = std::max<int64_t>(4, (int64_t)(share / 32.0));
+  const double over = 1.0 + share / 128.0;
+  for (int it = 0; it < 400 && assign(share, m, over) > slots; ++it) share *= 1.002;
+  if (assign(share, m, over) > slots) return false;
+  if ((int64_t)pieces.size() > kMaxItems) return false;
+  // workspace slots: consecutive for the parts of each cut row block, in row-block order
+  std::vector<int32_t> parts(n_rb, 0);
+  for (const Piece& pc : pieces) ++parts[pc.rb];
+  std::vector<int32_t> first(n_rb, -1);
+  Schedule sch;
+  sch.rows_per_block = per * kTileRows;
+  for (int64_t rb = 0; rb < n_rb; ++rb) {
+    if (parts[rb] > 1) {
+      first[rb] = sch.n_slots;
+      sch.split.push_back({(int32_t)rb, sch.n_slots, parts[rb], 0});
+      sch.n_slots += parts[rb];
+    }
+    sch.max_parts = std::max(sch.max_parts, parts[rb]);
+  }
+  if ((int64_t)sch.split.size() > kMaxSplitBlocks || sch.max_parts > PA_MAX_SPLITS) return false;
+  std::vector<int32_t> seen(n_rb, 0);
+  std::vector<std::pair<std::pair<double, int>, PaItem>> order;
+  for (const Piece& pc : pieces) {  // pieces of a row block appear in key order
+    const int32_t slot = parts[pc.rb] > 1 ? first[pc.rb] + seen[pc.rb]++ : -1;
+    order.push_back({{pc.start, pc.worker}, PaItem{pc.rb, pc.kt0, pc.kt1, slot}});
+  }
+  std::stable_sort(order.begin(), order.end(),
+                   [](const auto& x, const auto& y) { return x.first < y.first; });
+  for (const auto& o : order) sch.items.push_back(o.second);
+  double comb = 0.0;
+  if (!sch.split.empty()) {
+    double bytes = 0.0;
+    for (const PaSplitBlock& b : sch.split)
+      bytes += (double)(b.nparts + 1) * sch.rows_per_block * (p.head_dim + 1) * 4.0;
+    comb = bytes * cm.combine_us_per_byte + cm.combine_fixed_us;
+  }
+  sch.makespan_us = simulate_items(sch.items, slots, cm) + comb;
+  *out = std::move(sch);
+  return true;
+}
+
+}  // namespace pa
 
 extern "C" int pa_cores_policy_splits(int cores, int kv_heads, int tiles) {
   if (cores <= 0 || kv_heads <= 0 || tiles <= 0) return 1;
@@ -96,7 +222,7 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
   if (num_sms <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || chunk_rows <= 0 || hist_len < 0)
     return PA_ERR_INVALID_ARG;
   if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
-  if (splits_override < 0 || policy < 0 || policy > PA_POLICY_LEGACY) return PA_ERR_INVALID_ARG;
+  if (splits_override < 0 || policy < 0 || policy > PA_POLICY_BALANCED) return PA_ERR_INVALID_ARG;
   if (!(scale >= 0.0f) || isinf(scale)) return PA_ERR_INVALID_ARG;
   if (n_q_heads % n_kv_heads) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
@@ -115,7 +241,7 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
   const int64_t q_units = (q_tiles + per - 1) / per;
 
   int S = 1;
-  int used_policy = policy;
+  int used_policy = policy == PA_POLICY_BALANCED ? PA_POLICY_MAKESPAN : policy;
   if (splits_override > 0) {
     S = splits_override;
     used_policy = -1;
@@ -123,7 +249,7 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
     S = pa_cores_policy_splits(num_sms, n_kv_heads, (int)std::min<int64_t>(q_tiles, 1 << 30));
   } else if (policy == PA_POLICY_LEGACY) {
     S = pa_legacy_policy_splits(n_kv_heads, (int)std::min<int64_t>(q_tiles, 1 << 30));
-  } else {
+  } else {  // makespan, and the uniform candidate of the balanced policy
     double best = 0.0;
     const int64_t base_units = q_units * n_kv_heads;
     for (int cand = 1; cand <= PA_MAX_SPLITS; ++cand) {
@@ -160,7 +286,36 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
                                   head_dim) +
                          combine_cost(S, chunk_rows, n_q_heads, head_dim));
   plan->ws_bytes = S > 1 ? (uint64_t)S * chunk_rows * n_q_heads * (head_dim + 1) * 4ull : 0ull;
+
+  // The balanced schedule: always under the balanced policy (when it fits the kernel's
+  // tables), and under the makespan policy when its simulated time beats the best uniform one.
+  if (splits_override == 0 && (policy == PA_POLICY_BALANCED || policy == PA_POLICY_MAKESPAN)) {
+    pa::Schedule sch;
+    if (pa::build_balanced(*plan, &sch) &&
+        (policy == PA_POLICY_BALANCED || sch.makespan_us < plan->est_us * 0.99)) {
+      plan->policy = PA_POLICY_BALANCED;
+      plan->splits = sch.max_parts;
+      plan->units = (int64_t)sch.items.size();
+      plan->est_us = (float)sch.makespan_us;
+      plan->ws_bytes = (uint64_t)sch.n_slots * sch.rows_per_block * (head_dim + 1) * 4ull;
+    }
+  }
   return PA_OK;
+}
+
+extern "C" int pa_schedule_items(const pa_plan_t* plan, int32_t* items, int cap) {
+  if (!plan || plan->policy != PA_POLICY_BALANCED) return 0;
+  pa::Schedule sch;
+  if (!pa::build_balanced(*plan, &sch) || (int64_t)sch.items.size() != plan->units)
+    return PA_ERR_INVALID_ARG;
+  const int n = (int)sch.items.size();
+  for (int i = 0; i < n && i < cap && items; ++i) {
+    items[4 * i + 0] = sch.items[i].rb;
+    items[4 * i + 1] = sch.items[i].kt0;
+    items[4 * i + 2] = sch.items[i].kt1;
+    items[4 * i + 3] = sch.items[i].slot;
+  }
+  return n;
 }
 
 extern "C" const char* pa_status_string(int status) {

@@ -45,7 +45,8 @@ __device__ __forceinline__ uint32_t v_offset_pair(uint32_t k, uint32_t pl, int v
 template <bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a,
+                        const __grid_constant__ ItemTable items) {
   using C = PairCfg;
   constexpr int D = 256, NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
@@ -53,17 +54,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs, 1 relays
+  const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
+  PA_UNIT_ONLY(const uint64_t t_entry = globaltimer_ns();)
 
-  int64_t tp;
-  int g, s;
+  int64_t tp, kt0, kt1;
+  int g, s, slot = kSlotUniform;
   const int64_t q_pairs = (a.q_tiles + 1) / 2;
-  unit_coords(blockIdx.x >> 1, q_pairs, a.Hkv, a.splits, &tp, &g, &s);
+  if (a.balanced) {
+    const PaItem it = items.item[blockIdx.x >> 1];
+    rb_coords(it.rb, q_pairs, a.Hkv, &tp, &g);
+    s = 0;
+    kt0 = it.kt0;
+    kt1 = it.kt1;
+    slot = it.slot;
+  } else {
+    unit_coords(blockIdx.x >> 1, q_pairs, a.Hkv, a.splits, &tp, &g, &s);
+    const int64_t qt_last = 2 * tp + 1 < a.q_tiles ? 2 * tp + 1 : a.q_tiles - 1;
+    split_range(tile_kv_tiles(qt_last, a.R, a.G, a.hist_len), s, a.splits, &kt0, &kt1);
+  }
   const int64_t qt = 2 * tp + rank;
-  const int64_t qt_last = 2 * tp + 1 < a.q_tiles ? 2 * tp + 1 : a.q_tiles - 1;
-  const int64_t n_kt_all = tile_kv_tiles(qt_last, a.R, a.G, a.hist_len);
-  int64_t kt0, kt1;
-  split_range(n_kt_all, s, a.splits, &kt0, &kt1);
   const int n = (int)(kt1 - kt0);
 
   if (n == 0) {  // both CTAs of the pair see the same (empty) key range: empty partial
@@ -160,6 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.s = s;
     sc.kt0 = kt0;
     sc.n = n;
+    sc.slot = slot;
+    sc.row0 = (int)rank * kTileRows;
     sc.abort_flag = abort_flag;
     sc.tmo = tmo;
     // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
@@ -389,6 +400,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192) {
+    g_pa_units[4 * blockIdx.x + 0] = t_entry;
+    g_pa_units[4 * blockIdx.x + 1] = globaltimer_ns();
+    g_pa_units[4 * blockIdx.x + 2] = (uint64_t)n;
+    g_pa_units[4 * blockIdx.x + 3] = smid_u32();
+  })
   if (warp == kMmaWarp) {
     // The pair's tensor memory is freed only when both CTAs are done with it.
     if (lane == 0) mbar_arrive_remote(mapa_shared(bar(C::B_TEAR), rank ^ 1u));

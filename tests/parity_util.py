@@ -55,10 +55,10 @@ def custom_workload(name, Hq, Hkv, D, PS, dtype, pieces, seed, splits=0, pool_fa
                     splits=splits, scale=scale, seed_base=seed)
 
 
-def run_gpu(inp: Inputs, paged=True, splits=None, policy="makespan"):
+def run_gpu(inp: Inputs, paged=True, splits=None, policy="makespan", num_sms=None):
     from paged_kv_long_b200.runner import DeviceWorkload
     import torch
-    dw = DeviceWorkload(inp, "cuda", paged=paged, splits=splits, policy=policy)
+    dw = DeviceWorkload(inp, "cuda", paged=paged, splits=splits, policy=policy, num_sms=num_sms)
     dw.run()
     torch.cuda.synchronize()
     return dw, dw.outputs_host()

@@ -7,6 +7,7 @@ the oracle computes one by one. Tolerance: max-abs <= 1e-2 and relative RMS <= 2
 import numpy as np
 import pytest
 
+from paged_kv_long_b200 import binding
 from tests import parity_util as U
 from tests.conftest import cuda_available
 
@@ -93,6 +94,33 @@ def test_units_spanning_several_kv_tiles(idx):
     for paged in (True, False):
         _, outs = U.run_gpu(inp, paged=paged)
         U.check_full(inp, outs, paged=paged, what=f"{MULTI_TILE[idx]} paged={paged}")
+
+
+BALANCED = [
+    # Hq, Hkv, D, PS, dtype, pieces, num_sms: few SMs, so that row blocks are cut into parts
+    (24, 4, 256, 64, "bf16", [(3000, 100), (3100, 77)], 16),
+    (16, 2, 256, 16, "f16", [(5000, 40)], 6),
+    (16, 2, 256, 16, "f16", [(20000, 16)], 8),
+    (6, 2, 128, 32, "f16", [(1500, 131)], 6),
+    (4, 1, 64, 16, "bf16", [(2500, 99)], 3),
+    (4, 1, 64, 16, "f16", [(9000, 30)], 4),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(BALANCED)), ids=[f"b{i}" for i in range(len(BALANCED))])
+def test_balanced_schedule_full(idx):
+    """Work items that cut row blocks at arbitrary KV tiles (the balanced policy), merged by
+    the combine of cut row blocks; uncut row blocks write the output directly."""
+    Hq, Hkv, D, PS, dt, pieces, sms = BALANCED[idx]
+    wl = U.custom_workload("balanced", Hq, Hkv, D, PS, dt, pieces, seed=1300 + 10 * idx)
+    inp = U.gen(wl)
+    dw, outs = U.run_gpu(inp, policy="balanced", num_sms=sms)
+    assert all(p.policy == binding.PA_POLICY_BALANCED for p in dw.plans)
+    assert any((binding.schedule_items(p)[:, 3] >= 0).any() for p in dw.plans)
+    U.check_full(inp, outs, what=f"{BALANCED[idx]}")
+    _, outc = U.run_gpu(inp, paged=False, policy="balanced", num_sms=sms)
+    for a, b in zip(outs, outc):
+        assert np.array_equal(a, b)
 
 
 def test_online_rescale_with_growing_scores():
