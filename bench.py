@@ -319,11 +319,11 @@ def gpu_arm(args):
     t_contig = last_paged = last_contig = None
     if paged and not args.no_contiguous:
         from paged_kv_long_b200 import binding
-        dwc = DeviceWorkload(inp, dev, paged=False, splits=None, policy=args.policy)
-        for i, p in enumerate(dw.plans):   # same S per piece as the paged run
-            h, r = wl.pieces[i]
-            dwc.plans[i] = binding.plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size, r,
-                                        h, wl.dtype, wl.scale, p.splits, "makespan", False)
+        # the same schedule per piece as the paged run (the planner does not look at the layout)
+        dwc = DeviceWorkload(inp, dev, paged=False, splits=split_arg, policy=args.policy)
+        for p, pc in zip(dw.plans, dwc.plans):
+            assert (p.policy, p.splits, p.units, p.ws_bytes) == (pc.policy, pc.splits, pc.units,
+                                                                pc.ws_bytes)
         c_ms, c_kern = time_steps(dwc, max(3, args.steps // 2), args.warmup, flush, stream,
                                   record_kernels=True)
         t_contig = sum(c_ms) / len(c_ms)
@@ -373,7 +373,7 @@ def gpu_arm(args):
                      "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": None,
                      "peak_source": f"{peaks['source']} bf16 dense (burst)",
                      "step_frac_of_roofline": t_roof / (t_step / 1e3),
-                     "kernel": "prefill_kernel (pa_prefill)",
+                     "kernel": "prefill_pair_kernel (pa_prefill, head dim 256)" if wl.head_dim == 256 else "prefill_kernel (pa_prefill)",
                      "algorithmic_flops_per_step": flops},
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -394,7 +394,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="c5", choices=["c1", "c2", "c3", "c4", "c5"])
     ap.add_argument("--splits", type=int, default=None,
                     help="split count for every piece (default: the workload's, else the planner)")
-    ap.add_argument("--policy", default="makespan", choices=["makespan", "cores", "legacy"])
+    ap.add_argument("--policy", default="makespan", choices=["makespan", "cores", "legacy", "balanced"])
     ap.add_argument("--layout", default="paged", choices=["paged", "contiguous"])
     ap.add_argument("--no-contiguous", action="store_true", help="skip the contiguous control")
     ap.add_argument("--l2-flush-mb", type=int, default=L2_FLUSH_BYTES >> 20)

@@ -122,7 +122,8 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
 
 #ifdef PA_UNIT_TIMING
 // Instrumented builds only: per CTA (blockIdx < 8192) the global timer at entry and at exit,
-// its key-tile count and its SM (see pa_unit_timing).
+// its key-tile count with its SM in the upper half, and its SM clock cycles (see
+// pa_unit_timing).
 __device__ unsigned long long g_pa_units[4 * 8192];
 __device__ __forceinline__ uint32_t smid_u32() {
   uint32_t r;

@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
-  PA_UNIT_ONLY(const uint64_t t_entry = globaltimer_ns();)
+  PA_UNIT_ONLY(const uint64_t t_entry = globaltimer_ns(); const long long c_entry = clock64();)
 
   int64_t tp, kt0, kt1;
   int g, s, slot = kSlotUniform;
@@ -360,29 +360,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           PA_TRACE_ONLY(tlog(6, tln_w, 14, i);)
           ok = wait_cluster(bar(C::B_PFULL + (i & 1)), (i >> 1) & 1);
           PA_TRACE_ONLY(tlog(3, tln, 5, i);)
-          const uint32_t vslot0 = slot;
+          // Each half of the V tile (keys 0-63, then 64-127) is multiplied as soon as its slot
+          // has landed, and its slot is released right after its four MMAs.
+          const uint32_t p_tmem = tmem + kSCol0 + 128u * (i & 1) + kPColOff;
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
+          for (int h = 0; h < 2; ++h) {
             if (ok) ok = wait_slot();
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 4 * h; ks < 4 * h + 4; ++ks) {
+              const uint32_t off = v_offset_pair(16u * ks, 0, a.v_shift);
+              umma_ts_pair(tmem + kOCol, p_tmem + ks * 8,
+                           v_desc + slot * kSlotDesc + ((off & (kPanel - 1)) >> 4), idesc_pv,
+                           (i > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit_pair(bar(C::B_EMPTY + slot), kBoth);
             advance();
           }
           if (!ok) break;
           PA_TRACE_ONLY(tlog(3, tln, 6, round * NSLOT + slot - 2);)
-          tc_fence_after();
-          const uint32_t p_tmem = tmem + kSCol0 + 128u * (i & 1) + kPColOff;
-#pragma unroll
-          for (int ks = 0; ks < kTileKeys / 16; ++ks) {
-            const uint32_t off = v_offset_pair(16u * ks, 0, a.v_shift);
-            uint32_t vs = vslot0 + (off >> 14);
-            if (vs >= (uint32_t)NSLOT) vs -= NSLOT;
-            umma_ts_pair(tmem + kOCol, p_tmem + ks * 8,
-                         v_desc + vs * kSlotDesc + ((off & (kPanel - 1)) >> 4), idesc_pv,
-                         (i > 0 || ks > 0) ? 1u : 0u);
-          }
-          uint32_t vs1 = vslot0 + 1;
-          if (vs1 >= (uint32_t)NSLOT) vs1 -= NSLOT;
-          umma_commit_pair(bar(C::B_EMPTY + vslot0), kBoth);
-          umma_commit_pair(bar(C::B_EMPTY + vs1), kBoth);
           umma_commit_pair(bar(C::B_PVDONE + (i & 1)), kBoth);
           PA_TRACE_ONLY(tlog(3, tln, 7, i);)
         }
@@ -403,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192) {
     g_pa_units[4 * blockIdx.x + 0] = t_entry;
     g_pa_units[4 * blockIdx.x + 1] = globaltimer_ns();
-    g_pa_units[4 * blockIdx.x + 2] = (uint64_t)n;
-    g_pa_units[4 * blockIdx.x + 3] = smid_u32();
+    g_pa_units[4 * blockIdx.x + 2] = (uint64_t)n | ((uint64_t)smid_u32() << 32);
+    g_pa_units[4 * blockIdx.x + 3] = (uint64_t)(clock64() - c_entry);
   })
   if (warp == kMmaWarp) {
     // The pair's tensor memory is freed only when both CTAs are done with it.
