@@ -121,10 +121,12 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
 }
 
 #ifdef PA_UNIT_TIMING
-// Instrumented builds only: per CTA (blockIdx < 8192) the global timer at entry and at exit,
-// its key-tile count with its SM in the upper half, and its SM clock cycles (see
+// Instrumented builds only: per CTA (blockIdx < 8192) 8 words: the global timer at entry and
+// at exit, its key-tile count with its SM in the upper half, then SM clock readings at entry,
+// after set-up, when the first S tile was seen, when the epilogue began and at exit (see
 // pa_unit_timing).
-__device__ unsigned long long g_pa_units[4 * 8192];
+constexpr int kUnitWords = 8;
+__device__ unsigned long long g_pa_units[kUnitWords * 8192];
 __device__ __forceinline__ uint32_t smid_u32() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
@@ -218,6 +220,7 @@ struct SoftmaxCtx {
   int slot;       // workspace slot of a balanced item's partial, -1: final output,
                   // kSlotUniform: uniform splits (out when S == 1, else split s's partial)
   int row0;       // first packed row of this CTA inside its row block (balanced slots)
+  uint32_t stage_off;  // shared memory free once the last PV is done: 128 x (4D + 16) bytes
   volatile int* abort_flag;
   uint64_t tmo;
 };
@@ -280,6 +283,8 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       }
       PA_TRACE_ONLY(const long long tc = clock64(); tr[0] += tc - tw;
                     if (threadIdx.x == 0) tlog(5, tln, 8, j);)
+      PA_UNIT_ONLY(if (j == 0 && threadIdx.x == 0 && blockIdx.x < 8192)
+                       g_pa_units[kUnitWords * blockIdx.x + 5] = clock64();)
       tc_fence_after();
       float sv[kTileKeys];
 #pragma unroll
@@ -384,6 +389,8 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
     if (ok && n >= 2)
       ok = warp_wait(x.bar_pvdone + 8u * ((n - 2) & 1), ((n - 2) >> 1) & 1, abort_flag, tmo);
     if (ok) ok = warp_wait(x.bar_pvdone + 8u * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, tmo);
+    PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
+                     g_pa_units[kUnitWords * blockIdx.x + 6] = clock64();)
     if (ok) {
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -393,19 +400,25 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       else if (x.slot == kSlotUniform && a.splits > 1)
         ws_row = ((int64_t)s * a.R + tok) * a.Hq + head;
       float* dst = ws_row < 0 ? a.out + (tok * a.Hq + head) * (int64_t)D : a.ws_o + ws_row * D;
+      // The row goes through shared memory (the K/V ring, idle now; rows 16 bytes apart from
+      // a multiple of 128 so a warp's stores spread over the banks) and leaves as one
+      // contiguous bulk copy per row.
+      const uint32_t srow = sb + x.stage_off + (uint32_t)r * (uint32_t)(D * 4 + 16);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
         tmem_ld32(t_lane + kOCol + 32u * c, o);
         tmem_wait_ld();
-        if (valid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(o[4 * i] * inv_l, o[4 * i + 1] * inv_l, o[4 * i + 2] * inv_l,
-                                o[4 * i + 3] * inv_l);
-        }
+        for (int i = 0; i < 8; ++i)
+          st_shared_v4(srow + 128u * c + 16u * i, __float_as_uint(o[4 * i] * inv_l),
+                       __float_as_uint(o[4 * i + 1] * inv_l), __float_as_uint(o[4 * i + 2] * inv_l),
+                       __float_as_uint(o[4 * i + 3] * inv_l));
       }
+      fence_proxy_async_smem();
+      if (valid) bulk_store(dst, srow, D * 4);
+      bulk_commit();
+      bulk_wait_read_all();
       if (valid && ws_row >= 0) a.ws_lse[ws_row] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
     }
     PA_TRACE_ONLY(tr[2] += clock64() - te;
@@ -518,6 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.n = n;
     sc.slot = slot;
     sc.row0 = 0;
+    sc.stage_off = C::RING_OFF;
+    static_assert(C::NSLOT * kPanel >= kTileRows * (D * 4 + 16), "staging needs the ring");
     sc.abort_flag = abort_flag;
     sc.tmo = tmo;
     // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
@@ -1149,10 +1164,10 @@ extern "C" int pa_device_error(int* flags, int reset) {
 #ifdef PA_UNIT_TIMING
 extern "C" int pa_unit_timing(unsigned long long* out, int cap, int reset) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  int n = cap < 4 * 8192 ? cap : 4 * 8192;
+  int n = cap < kUnitWords * 8192 ? cap : kUnitWords * 8192;
   if (cudaMemcpyFromSymbol(out, g_pa_units, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
   if (reset) {
-    static unsigned long long z[4 * 8192];
+    static unsigned long long z[kUnitWords * 8192];
     cudaMemcpyToSymbol(g_pa_units, z, sizeof z);
   }
   return n;

@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
+  PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
+                   g_pa_units[kUnitWords * blockIdx.x + 4] = clock64();)
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
   PA_TRACE_ONLY(unsigned tln = 0;)
@@ -171,6 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.n = n;
     sc.slot = slot;
     sc.row0 = (int)rank * kTileRows;
+    sc.stage_off = C::RING_OFF;
+    static_assert(NSLOT * kPanel >= kTileRows * (D * 4 + 16), "staging needs the ring");
     sc.abort_flag = abort_flag;
     sc.tmo = tmo;
     // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
@@ -398,10 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192) {
-    g_pa_units[4 * blockIdx.x + 0] = t_entry;
-    g_pa_units[4 * blockIdx.x + 1] = globaltimer_ns();
-    g_pa_units[4 * blockIdx.x + 2] = (uint64_t)n | ((uint64_t)smid_u32() << 32);
-    g_pa_units[4 * blockIdx.x + 3] = (uint64_t)(clock64() - c_entry);
+    unsigned long long* u = g_pa_units + kUnitWords * blockIdx.x;
+    u[0] = t_entry;
+    u[1] = globaltimer_ns();
+    u[2] = (uint64_t)n | ((uint64_t)smid_u32() << 32);
+    u[3] = (uint64_t)c_entry;
+    u[7] = (uint64_t)clock64();
   })
   if (warp == kMmaWarp) {
     // The pair's tensor memory is freed only when both CTAs are done with it.
