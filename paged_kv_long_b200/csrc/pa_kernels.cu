@@ -27,6 +27,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <cstring>
 #include <atomic>
 #include <mutex>
 
@@ -72,6 +73,7 @@ struct PrefillArgs {
   int32_t oob_row;       // a key-row coordinate past the pool: the TMA fills zeros there
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
+  int32_t q_tma;           // 1: the Q tile arrives by tensor copy (CTA-pair kernel, G | 128)
   int32_t balanced;        // 1: CTA (pair) b runs work item b of the item table
   int32_t rows_per_block;  // packed rows of a row block (balanced workspace slots)
 };
@@ -121,11 +123,12 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
 }
 
 #ifdef PA_UNIT_TIMING
-// Instrumented builds only: per CTA (blockIdx < 8192) 8 words: the global timer at entry and
+// Instrumented builds only: per CTA (blockIdx < 8192) 12 words: the global timer at entry and
 // at exit, its key-tile count with its SM in the upper half, then SM clock readings at entry,
-// after set-up, when the first S tile was seen, when the epilogue began and at exit (see
-// pa_unit_timing).
-constexpr int kUnitWords = 8;
+// after set-up, when the first S tile was seen, when the epilogue began, at exit, when the MMA
+// warp saw Q, when it saw the first K slot, when the Q tile was stored, and when the first
+// K/V copy was issued (see pa_unit_timing).
+constexpr int kUnitWords = 12;
 __device__ unsigned long long g_pa_units[kUnitWords * 8192];
 __device__ __forceinline__ uint32_t smid_u32() {
   uint32_t r;
@@ -248,8 +251,9 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
     const int64_t tok = grow / a.G;
     const bool valid = tok < a.R;
     const int head = g * a.G + (int)(grow % a.G);
-    {
-      // Q tile -> shared memory as K-major rows of 64-element panels, 128-byte swizzle.
+    if (!a.q_tma) {
+      // Q tile -> shared memory as K-major rows of 64-element panels, 128-byte swizzle (when
+      // the tensor copy cannot: it loads whole tokens, so it needs G to divide 128).
       const uint4* src =
           reinterpret_cast<const uint4*>(a.q + (valid ? (tok * a.Hq + head) * (int64_t)D : 0));
 #pragma unroll
@@ -263,6 +267,8 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       }
       fence_proxy_async_smem();
       __syncwarp();
+      PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
+                       g_pa_units[kUnitWords * blockIdx.x + 10] = clock64();)
       if (lane == 0) arrive(x.arrive_qfull);
     }
 
@@ -894,6 +900,25 @@ bool make_v_map(CUtensorMap* map, const void* base, bool bf16, int D, int Hkv, i
   return r == CUDA_SUCCESS;
 }
 
+// Q of one piece as a 4-D tensor {D, G, Hkv, R}: a box is 64 elements (one swizzle row) of
+// all G heads of KV head g for 128/G tokens, i.e. one panel of a packed 128-row Q tile when
+// G divides 128. Rows past the piece read as zeros.
+bool make_q_map(CUtensorMap* map, const void* base, bool bf16, int D, int G, int Hkv, int R) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)G, (cuuint64_t)Hkv, (cuuint64_t)R};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)G * D * 2,
+                                 (cuuint64_t)Hkv * G * D * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)(kTileRows / G)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r =
+      fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, bool PAGED, bool BF16>
 cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
                            const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
@@ -915,7 +940,8 @@ cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
 
 template <bool PAGED, bool BF16>
 cudaError_t launch_pair(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
-                        const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
+                        const CUtensorMap& tv, const CUtensorMap& tq, const PrefillArgs& a,
+                        const ItemTable& it) {
   auto kern = prefill_pair_kernel<PAGED, BF16>;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -940,7 +966,7 @@ cudaError_t launch_pair(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a, it);
+  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, a, it);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1013,6 +1039,12 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows) ||
       !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, v_panels))
     return PA_ERR_CUDA;
+  // CTA pair: Q by tensor copy when a packed 128-row tile is whole tokens
+  CUtensorMap tq;
+  const bool q_tma = per == 2 && kTileRows % plan->group == 0;
+  if (q_tma && !make_q_map(&tq, q, bf16, D, plan->group, plan->n_kv_heads, chunk_rows))
+    return PA_ERR_CUDA;
+  if (!q_tma) memset(&tq, 0, sizeof tq);
 
   PrefillArgs a;
   a.q = static_cast<const uint16_t*>(q);
@@ -1042,6 +1074,7 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.scale_log2 = plan->scale * 1.4426950408889634f;
   a.timeout_ns = g_timeout_ns.load();
   a.balanced = balanced ? 1 : 0;
+  a.q_tma = q_tma ? 1 : 0;
   a.rows_per_block = per * kTileRows;
   // Kernel parameter of 8 KB, copied into the launch: kept off the stack of callers with small
   // stacks, one per thread (the launch has taken its copy when this function returns).
@@ -1055,10 +1088,10 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
     case 64: e = launch_d<64>(paged, bf16, grid, st, tk, tv, a, *tab); break;
     case 128: e = launch_d<128>(paged, bf16, grid, st, tk, tv, a, *tab); break;
     default:
-      e = paged ? (bf16 ? launch_pair<true, true>(grid, st, tk, tv, a, *tab)
-                        : launch_pair<true, false>(grid, st, tk, tv, a, *tab))
-                : (bf16 ? launch_pair<false, true>(grid, st, tk, tv, a, *tab)
-                        : launch_pair<false, false>(grid, st, tk, tv, a, *tab));
+      e = paged ? (bf16 ? launch_pair<true, true>(grid, st, tk, tv, tq, a, *tab)
+                        : launch_pair<true, false>(grid, st, tk, tv, tq, a, *tab))
+                : (bf16 ? launch_pair<false, true>(grid, st, tk, tv, tq, a, *tab)
+                        : launch_pair<false, false>(grid, st, tk, tv, tq, a, *tab));
       break;
   }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -45,7 +45,8 @@ __device__ __forceinline__ uint32_t v_offset_pair(uint32_t k, uint32_t pl, int v
 template <bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_q, const PrefillArgs a,
                         const __grid_constant__ ItemTable items) {
   using C = PairCfg;
   constexpr int D = 256, NSLOT = C::NSLOT;
@@ -107,7 +108,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::B_FULL + i), 1);
       mbar_init(bar(C::B_EMPTY + i), 1);
     }
-    mbar_init(bar(C::B_QFULL), 8);   // 4 warps here + 4 warps of rank 1
+    // Q by tensor copy: one arrival (rank 0's, with both CTAs' bytes); else 4 softmax warps
+    // here + 4 of rank 1
+    mbar_init(bar(C::B_QFULL), a.q_tma ? 1 : 8);
     mbar_init(bar(C::B_SFULL + 0), 1);
     mbar_init(bar(C::B_SFULL + 1), 1);
     mbar_init(bar(C::B_PFULL + 0), 8);
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp + 1 && lane == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (a.q_tma) tma_prefetch_desc(&tm_q);
   }
   if (warp == kMmaWarp) {
     tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
@@ -250,6 +254,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto own_barrier = [&](uint32_t q) -> bool { return rank == 0 || tail_fill(q); };
     int32_t row_prev = a.oob_row, row_cur = fetch(0), row_next = fetch(1);
+    // Q tile: four 16 KB panels of 128/G whole tokens; both CTAs' bytes complete on rank 0's
+    // barrier, which rank 0 arms for both. Rows past the piece arrive as zeros.
+    if (a.q_tma && w == 0 && lane == 0) {
+      const int32_t t0 = (int32_t)(qt * (kTileRows / a.G));
+      if (rank == 0) mbar_arrive_expect_tx(bar(C::B_QFULL), 2u * 4u * kPanel);
+      for (int p = 0; p < 4; ++p) {
+        if (rank == 0)
+          tma_load_4d(sb + C::Q_OFF + p * kPanel, &tm_q, bar(C::B_QFULL), p * 64, 0, g, t0);
+        else
+          tma_load_4d_pair(sb + C::Q_OFF + p * kPanel, &tm_q, leader_bar(C::B_QFULL), p * 64, 0,
+                           g, t0);
+      }
+    }
     uint32_t issued_end = 0;
     for (int j = 0; j <= n && ok; ++j) {
       if (j < n) {  // K half tile j: slot k holds panels 2k, 2k+1 of keys 64*rank..+63
@@ -270,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                row);
           }
           issued_end = q + 1;
+          PA_UNIT_ONLY(if (q == 0 && lane == 0 && blockIdx.x < 8192)
+                           g_pa_units[kUnitWords * blockIdx.x + 11] = clock64();)
           PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 1, q);)
         }
       }
@@ -333,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       bool ok = wait_cluster(bar(C::B_QFULL), 0);
+      PA_UNIT_ONLY(if (blockIdx.x < 8192) g_pa_units[kUnitWords * blockIdx.x + 8] = clock64();)
       tc_fence_after();
       for (int j = 0; j <= n && ok; ++j) {
         if (j < n) {
@@ -340,6 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             if (!(ok = wait_slot())) break;
+            PA_UNIT_ONLY(if (j == 0 && k == 0 && blockIdx.x < 8192)
+                             g_pa_units[kUnitWords * blockIdx.x + 9] = clock64();)
             PA_TRACE_ONLY(tlog(3, tln, 3, round * NSLOT + slot);)
             tc_fence_after();
 #pragma unroll
