@@ -126,9 +126,10 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
 // Instrumented builds only: per CTA (blockIdx < 8192) 12 words: the global timer at entry and
 // at exit, its key-tile count with its SM in the upper half, then SM clock readings at entry,
 // after set-up, when the first S tile was seen, when the epilogue began, at exit, when the MMA
-// warp saw Q, when it saw the first K slot, when the Q tile was stored, and when the first
-// K/V copy was issued (see pa_unit_timing).
-constexpr int kUnitWords = 12;
+// warp saw Q, when it saw the first K slot, when the Q tile was stored, when the first K/V copy
+// was issued, and the MMA lane's cycles waiting for K slots, V slots and P (see
+// pa_unit_timing).
+constexpr int kUnitWords = 16;
 __device__ unsigned long long g_pa_units[kUnitWords * 8192];
 __device__ __forceinline__ uint32_t smid_u32() {
   uint32_t r;

@@ -24,16 +24,17 @@ namespace {
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
-// Cost model (microseconds), B200: a 128x128 KV tile costs 4*128*128*D FLOPs at about
-// 1.4 PFLOP/s shared by 148 SMs; a unit pays a fixed start/finish cost (tensor memory
-// allocation, Q tile load, pipeline fill, writing 128 rows of fp32 output); the combine
-// streams S partials through HBM.
+// Cost model (microseconds), B200, fitted to the kernels' measured cycle counts (regression
+// over items of 4-256 tiles at ~1.7 GHz, head dim 256): a 128x128 KV tile costs 4*128*128*D
+// FLOPs at about 1.5 PFLOP/s shared by 148 SMs; a unit pays a fixed start/finish cost (set-up,
+// Q tile load and pipeline fill, writing 128 rows of fp32 output: ~13,000 cycles at D = 256);
+// the combine streams the partials through HBM.
 struct CostModel {
   double tile_us, unit_us, combine_us_per_byte, combine_fixed_us;
   explicit CostModel(int D) {
-    const double per_sm_flops = 1.4e15 / 148.0;
+    const double per_sm_flops = 1.5e15 / 148.0;
     tile_us = 4.0 * pa::kTileKeys * pa::kTileRows * D / per_sm_flops * 1e6;
-    unit_us = 2.0 + pa::kTileRows * (double)D * 4.0 / 60e9 * 1e6;
+    unit_us = 3.0 + pa::kTileRows * (double)D * 4.0 / 30e9 * 1e6;
     combine_us_per_byte = 1.0 / 5.0e12 * 1e6;
     combine_fixed_us = 4.0;
   }

@@ -341,9 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       PA_TRACE_ONLY(unsigned tln_w = 0;)
       // a slot is ready when both halves landed (one barrier; for the tail fills rank 1's half
       // is covered by its softmax warps' P-ready arrival, which waits for it)
+      PA_UNIT_ONLY(long long w_k = 0, w_v = 0, w_p = 0; long long* w_sel = &w_k;)
       auto wait_slot = [&]() -> bool {
         PA_TRACE_ONLY(tlog(6, tln_w, 11, round * NSLOT + slot);)
-        return thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
+        PA_UNIT_ONLY(const long long c0 = clock64();)
+        const bool r = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
+        PA_UNIT_ONLY(*w_sel += clock64() - c0;)
+        return r;
       };
       auto advance = [&]() {
         if (++slot == (uint32_t)NSLOT) {
@@ -359,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t s_tmem = tmem + kSCol0 + 128u * (j & 1);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
+            PA_UNIT_ONLY(w_sel = &w_k;)
             if (!(ok = wait_slot())) break;
             PA_UNIT_ONLY(if (j == 0 && k == 0 && blockIdx.x < 8192)
                              g_pa_units[kUnitWords * blockIdx.x + 9] = clock64();)
@@ -384,7 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1) {
           const int i = j - 1;
           PA_TRACE_ONLY(tlog(6, tln_w, 14, i);)
+          PA_UNIT_ONLY(const long long c0 = clock64();)
           ok = wait_cluster(bar(C::B_PFULL + (i & 1)), (i >> 1) & 1);
+          PA_UNIT_ONLY(w_p += clock64() - c0; w_sel = &w_v;)
           PA_TRACE_ONLY(tlog(3, tln, 5, i);)
           // Each half of the V tile (keys 0-63, then 64-127) is multiplied as soon as its slot
           // has landed, and its slot is released right after its four MMAs.
@@ -410,6 +417,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           PA_TRACE_ONLY(tlog(3, tln, 7, i);)
         }
       }
+      PA_UNIT_ONLY(if (blockIdx.x < 8192) {
+        g_pa_units[kUnitWords * blockIdx.x + 12] = (unsigned long long)w_k;
+        g_pa_units[kUnitWords * blockIdx.x + 13] = (unsigned long long)w_v;
+        g_pa_units[kUnitWords * blockIdx.x + 14] = (unsigned long long)w_p;
+      })
       umma_commit_pair(bar(C::B_MMADONE), kBoth);
       drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
     }
