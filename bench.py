@@ -223,6 +223,51 @@ def time_steps(dw, steps, warmup, flush, stream, record_kernels=False):
     return step_ms, kern_ms
 
 
+def kv_append_measure(inp, dev, stream, peaks, reps=20):
+    """pa_kv_append on the workload's rows: all of them in one call (HBM-bound; the roofline is
+    the measured copy bandwidth), and chunk by chunk as a prefill engine issues them."""
+    import numpy as np
+    import torch
+    from paged_kv_long_b200 import binding
+    wl = inp.wl
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+
+    def dev_bits(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(dt)
+
+    h0 = wl.first_pos
+    rows = wl.total_keys - h0
+    kn, vn = dev_bits(inp.k_logical[h0:h0 + rows]), dev_bits(inp.v_logical[h0:h0 + rows])
+    kp, vp = dev_bits(inp.k_pool), dev_bits(inp.v_pool)
+    tab = torch.from_numpy(inp.page_table).to(dev)
+    with torch.cuda.stream(stream):
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        t_all = timed(lambda: binding.kv_append(kn, vn, kp, vp, tab, h0, stream))
+
+        def chunks():
+            for h, r in wl.pieces:
+                binding.kv_append(kn[h - h0:h - h0 + r], vn[h - h0:h - h0 + r], kp, vp, tab, h,
+                                  stream)
+        t_chunks = timed(chunks)
+    nbytes = 2 * rows * wl.n_kv_heads * wl.head_dim * 2 * 2   # K and V, read once, written once
+    gbs = nbytes / (t_all * 1e-3) / 1e9
+    return {"workload": f"{rows} rows of K and V (all the workload's positions) in one call",
+            "ms": t_all, "GB_per_s": gbs, "peak_GB_per_s": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes,
+            "us_per_chunk_call_host_bound": t_chunks * 1e3 / len(wl.pieces),
+            "chunk_calls": len(wl.pieces)}
+
+
 def e2e_steps(inp, dw, steps, stream):
     """End to end through the public API: pinned host inputs -> device, prefill + combine for
     every piece, outputs -> pinned host, every step. Returns (per-step ms, h2d, d2h bytes)."""
@@ -331,6 +376,11 @@ def gpu_arm(args):
         last_contig = statistics.median(k[-1] for k in c_kern)
         del dwc
 
+    # ---- KV append, the step before prefill (its own HBM roofline)
+    kv = None
+    if paged and not args.no_kv_append:
+        kv = kv_append_measure(inp, dev, stream, peaks)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e and paged:
@@ -376,6 +426,7 @@ def gpu_arm(args):
                      "kernel": "prefill_pair_kernel (pa_prefill, head dim 256)" if wl.head_dim == 256 else "prefill_kernel (pa_prefill)",
                      "algorithmic_flops_per_step": flops},
         "e2e": e2e,
+        "kv_append": kv,
         "cpu_baseline": cpu,
         "gpu_launches": launches,
         "clocks": clocks,
@@ -399,6 +450,7 @@ def main(argv=None):
     ap.add_argument("--no-contiguous", action="store_true", help="skip the contiguous control")
     ap.add_argument("--l2-flush-mb", type=int, default=L2_FLUSH_BYTES >> 20)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-kv-append", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)

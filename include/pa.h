@@ -207,6 +207,24 @@ int pa_prefill_noalloc(const pa_plan_t* plan, const void* q, const void* k_pool,
                        int64_t hist_len, int chunk_rows, float* out, pa_stream_t stream);
 
 /*
+ * pa_kv_append — write a chunk's new K and V rows into the paged pools through the page table,
+ * enqueued on `stream`: the step before pa_prefill (BaseRT issue #51, "Results": the chunk's
+ * K/V are published to pages and prefill reads every key, its own included, through the table).
+ *   k_new, v_new   device [R][Hkv][D] of dtype, contiguous, 16-byte aligned.
+ *   k_pool, v_pool device [num_pages][PS][Hkv][D] (as pa_prefill), 16-byte aligned.
+ *   page_table     device int32 [ceil((H+R)/PS)]; hist_len H: position of the first new row;
+ *                  chunk_rows R (0: nothing to do).
+ * Row i goes to page page_table[(H+i)/PS], slot (H+i)%PS, all Hkv heads at once; nothing else
+ * in the pools changes. An entry outside [0, num_pages) skips its rows and raises
+ * PA_ERR_PAGE_INDEX in pa_device_error. Returns PA_OK, PA_ERR_INVALID_ARG,
+ * PA_ERR_UNSUPPORTED (head_dim not 64/128/256, page_size not a power of two in 16..128) or
+ * PA_ERR_CUDA.
+ */
+int pa_kv_append(int n_kv_heads, int head_dim, int page_size, int dtype, const void* k_new,
+                 const void* v_new, void* k_pool, void* v_pool, const int32_t* page_table,
+                 int64_t num_pages, int64_t hist_len, int chunk_rows, pa_stream_t stream);
+
+/*
  * pa_device_error — synchronise the current device, then read (and with reset != 0,
  * clear) the library's device-side error word. *flags receives its bits
  * (1: page index out of range, 2: a wait timed out). Returns PA_OK when no bit is set,

@@ -22,7 +22,7 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "P
 EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_device_error",
             "pa_set_wait_timeout_ns",
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
-            "pa_legacy_policy_splits", "pa_schedule_items")
+            "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append")
 
 
 class PaError(RuntimeError):
@@ -86,6 +86,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_legacy_policy_splits.restype = i32
     lib.pa_schedule_items.argtypes = [ctypes.POINTER(Plan), ctypes.POINTER(ctypes.c_int32), i32]
     lib.pa_schedule_items.restype = i32
+    lib.pa_kv_append.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i64, i32, vp]
+    lib.pa_kv_append.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -130,6 +132,33 @@ def schedule_items(p: Plan):
     buf = (ctypes.c_int32 * max(4 * n, 1))()
     lib.pa_schedule_items(ctypes.byref(p), buf, n)
     return np.frombuffer(buf, dtype=np.int32)[:4 * n].reshape(n, 4).copy()
+
+
+def kv_append(k_new, v_new, k_pool, v_pool, page_table, hist_len: int, stream=None):
+    """pa_kv_append: write the chunk's K/V rows [R, Hkv, D] into the page pools
+    [num_pages, PS, Hkv, D] at positions hist_len.. through page_table (see include/pa.h)."""
+    import torch
+    if k_new.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("k_new must be float16 or bfloat16")
+    dt = k_new.dtype
+    _require_cuda(k_new, "k_new", dt)
+    if k_new.dim() != 3:
+        raise ValueError("k_new must be [R, Hkv, D]")
+    R, Hkv, D = k_new.shape
+    _require_cuda(v_new, "v_new", dt, (R, Hkv, D))
+    _require_cuda(k_pool, "k_pool", dt)
+    if k_pool.dim() != 4 or tuple(k_pool.shape[2:]) != (Hkv, D):
+        raise ValueError("k_pool must be [num_pages, page_size, Hkv, D]")
+    _require_cuda(v_pool, "v_pool", dt, tuple(k_pool.shape))
+    _require_cuda(page_table, "page_table", torch.int32)
+    PS = k_pool.shape[1]
+    if page_table.numel() < math.ceil((hist_len + R) / PS):
+        raise ValueError("page_table is shorter than ceil((hist_len+R)/page_size)")
+    st = load_library().pa_kv_append(Hkv, D, PS, _dtype_code(dt), k_new.data_ptr(),
+                                     v_new.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                     page_table.data_ptr(), k_pool.shape[0], hist_len, R,
+                                     _stream_ptr(stream))
+    _check(st, "pa_kv_append")
 
 
 def _stream_ptr(stream):

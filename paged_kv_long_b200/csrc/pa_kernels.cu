@@ -745,6 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 #include "prefill_pair.cuh"
+#include "kv_append.cuh"
 
 // ---------------------------------------------------------------- combine kernel
 // One warp per (row, head): lanes hold the S <= 32 split LSEs, the warp reduces max and sum
@@ -1178,6 +1179,30 @@ extern "C" int pa_prefill_noalloc(const pa_plan_t* plan, const void* q, const vo
                             out, ws, ws_bytes, stream);
   if (st != PA_OK) return st;
   return pa_combine(plan, ws, ws_bytes, out, stream);
+}
+
+extern "C" int pa_kv_append(int n_kv_heads, int head_dim, int page_size, int dtype,
+                            const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                            const int32_t* page_table, int64_t num_pages, int64_t hist_len,
+                            int chunk_rows, pa_stream_t stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (n_kv_heads <= 0 || hist_len < 0 || chunk_rows < 0 || num_pages <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (page_size < 16 || page_size > 128 || (page_size & (page_size - 1))) return PA_ERR_UNSUPPORTED;
+  if (chunk_rows == 0) return PA_OK;
+  if (!k_new || !v_new || !k_pool || !v_pool || !page_table) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return PA_ERR_INVALID_ARG;
+  const int row_vecs = n_kv_heads * head_dim * 2 / 16;
+  const int64_t warps = 2 * (int64_t)chunk_rows;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  kv_append_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), page_table, num_pages, hist_len,
+      chunk_rows, page_size, row_vecs);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" int pa_device_error(int* flags, int reset) {
