@@ -246,6 +246,18 @@ int pa_selftest_timeout(uint64_t timeout_ns, pa_stream_t stream);
 /* pa_status_string — static description of a status code. */
 const char* pa_status_string(int status);
 
+/*
+ * pa_pieces — cut a chunk of chunk_rows query rows at history hist_len into pieces the way the
+ * pages' engine does at long context (splash PR #33, "What changed": 512 rows from 32K history,
+ * 256 from 64K, 128 past about 128K, per rows * (history + rows) <= 2^25): each piece is the
+ * largest power of two r of the rows left with r * (history + r) <= 2^log2_budget (at least one
+ * row), and each piece's history includes the pieces before it. Writes at most `cap` piece sizes
+ * (rows_out may be NULL) and returns the number of pieces, or PA_ERR_INVALID_ARG. Pure host code.
+ * On B200 the balanced planner fills the GPU without cutting chunks; the rule is kept to
+ * reproduce the pages' pieces (the 32K-history workload of four 512-row pieces).
+ */
+int pa_pieces(int chunk_rows, int64_t hist_len, int log2_budget, int32_t* rows_out, int cap);
+
 /* pa_cores_policy_splits — the split rule of splash PR #33 ("What changed") for a GPU with
  * `cores` cores, `kv_heads` KV heads and `tiles` tiles per KV head. Pure host function. */
 int pa_cores_policy_splits(int cores, int kv_heads, int tiles);

@@ -22,7 +22,7 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "P
 EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_device_error",
             "pa_set_wait_timeout_ns",
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
-            "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append")
+            "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append", "pa_pieces")
 
 
 class PaError(RuntimeError):
@@ -88,6 +88,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_schedule_items.restype = i32
     lib.pa_kv_append.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i64, i32, vp]
     lib.pa_kv_append.restype = i32
+    lib.pa_pieces.argtypes = [i32, i64, i32, ctypes.POINTER(ctypes.c_int32), i32]
+    lib.pa_pieces.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -132,6 +134,16 @@ def schedule_items(p: Plan):
     buf = (ctypes.c_int32 * max(4 * n, 1))()
     lib.pa_schedule_items(ctypes.byref(p), buf, n)
     return np.frombuffer(buf, dtype=np.int32)[:4 * n].reshape(n, 4).copy()
+
+
+def pieces(chunk_rows: int, hist_len: int, log2_budget: int = 25) -> list[int]:
+    """pa_pieces: the pages' cut of a chunk into pieces (rows of each, in order)."""
+    lib = load_library()
+    n = lib.pa_pieces(chunk_rows, hist_len, log2_budget, None, 0)
+    _check(0 if n >= 0 else n, "pa_pieces")
+    buf = (ctypes.c_int32 * max(n, 1))()
+    lib.pa_pieces(chunk_rows, hist_len, log2_budget, buf, n)
+    return list(buf)[:n]
 
 
 def kv_append(k_new, v_new, k_pool, v_pool, page_table, hist_len: int, stream=None):

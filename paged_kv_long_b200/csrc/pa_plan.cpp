@@ -204,6 +204,25 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
 
 }  // namespace pa
 
+extern "C" int pa_pieces(int chunk_rows, int64_t hist_len, int log2_budget, int32_t* rows_out,
+                         int cap) {
+  if (chunk_rows < 0 || hist_len < 0 || log2_budget < 1 || log2_budget > 62 || cap < 0)
+    return PA_ERR_INVALID_ARG;
+  const int64_t budget = int64_t(1) << log2_budget;
+  int n = 0;
+  int64_t h = hist_len, left = chunk_rows;
+  while (left > 0) {
+    // the largest power of two r <= left with r * (h + r) <= budget (at least one row)
+    int64_t r = 1;
+    while (2 * r <= left && 2 * r * (h + 2 * r) <= budget) r *= 2;
+    if (rows_out && n < cap) rows_out[n] = (int32_t)r;
+    ++n;
+    h += r;
+    left -= r;
+  }
+  return n;
+}
+
 extern "C" int pa_cores_policy_splits(int cores, int kv_heads, int tiles) {
   if (cores <= 0 || kv_heads <= 0 || tiles <= 0) return 1;
   const int target = std::min(256, std::max(32, (32 * cores) / kv_heads));

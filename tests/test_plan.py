@@ -135,3 +135,28 @@ def test_policies_selectable(lib):
 def test_status_strings(lib):
     for code in binding.STATUS:
         assert lib.pa_status_string(code)
+
+
+# ------------------------------------------------------------------ the pages' piece rule
+def test_pieces_reproduce_the_pages_sizes(lib):
+    # splash PR #33, "What changed": 512 rows from 32K history, 256 from 64K, 128 past ~128K
+    assert binding.pieces(2048, 32768)[0] == 512
+    assert binding.pieces(2048, 65536)[0] == 256
+    assert binding.pieces(2048, 131072)[0] == 128
+    # the 32K-history workload: four 512-row pieces
+    assert binding.pieces(2048, 32768) == [512, 512, 512, 512]
+
+
+@pytest.mark.parametrize("rows,hist", [(2048, 0), (2048, 30000), (1000, 100000), (7, 5),
+                                       (2048, 300000), (1, 0), (0, 10)])
+def test_pieces_cover_the_chunk_and_are_maximal(lib, rows, hist):
+    ps = binding.pieces(rows, hist)
+    assert sum(ps) == rows
+    h, left = hist, rows
+    for r in ps:
+        assert r >= 1 and (r & (r - 1)) == 0
+        assert r == 1 or r * (h + r) <= 1 << 25
+        # doubling would break the budget or run past the chunk
+        assert 2 * r > left or 2 * r * (h + 2 * r) > 1 << 25
+        h += r
+        left -= r
