@@ -268,6 +268,61 @@ def kv_append_measure(inp, dev, stream, peaks, reps=20):
             "chunk_calls": len(wl.pieces)}
 
 
+DECODE_BATCH = 32          # sequences of one decode step
+DECODE_LENS = (1024, 32768)  # key counts drawn uniformly from this range (the prompt sweep's)
+
+
+def decode_measure(wl, dev, stream, peaks, reps=20, seed=6000):
+    """pa_decode (+ pa_combine) on a batch of sequences over one shared page pool, with the
+    workload's heads, head dim, page size and dtype: HBM-bound (every key's K and V row read
+    once), so the roofline is the measured copy bandwidth."""
+    import numpy as np
+    import torch
+    from paged_kv_long_b200 import binding
+    from paged_kv_long_b200.inputs import decode_batch
+    lens = np.random.default_rng(seed).integers(DECODE_LENS[0], DECODE_LENS[1] + 1,
+                                               size=DECODE_BATCH)
+    db = decode_batch(seed + 1, lens, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size,
+                      wl.dtype, poison=False)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+
+    def dev_bits(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(dt)
+
+    q, kp, vp = dev_bits(db.q), dev_bits(db.k_pool), dev_bits(db.v_pool)
+    tab = torch.from_numpy(db.block_table).to(dev)
+    sl = torch.from_numpy(db.seq_lens).to(dev)
+    p = binding.decode_plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size,
+                            DECODE_BATCH, int(lens.max()), wl.dtype)
+    out = torch.empty((DECODE_BATCH, wl.n_q_heads, wl.head_dim), dtype=torch.float32,
+                      device=dev)
+    ws = binding.workspace(p, dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            binding.decode(p, q, kp, vp, tab, sl, out, ws, stream)
+        evs = []
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binding.decode(p, q, kp, vp, tab, sl, out, ws, stream)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    keys = int(lens.sum())
+    nbytes = (2 * keys * wl.n_kv_heads * wl.head_dim * 2            # K and V rows
+              + DECODE_BATCH * wl.n_q_heads * wl.head_dim * (2 + 4))  # Q in, fp32 out
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"{DECODE_BATCH} sequences, {keys} keys in all (lengths uniform in "
+                        f"{DECODE_LENS[0]}..{DECODE_LENS[1]}), one query token each, "
+                        f"{wl.n_q_heads}q/{wl.n_kv_heads}kv D{wl.head_dim} PS{wl.page_size} "
+                        f"{wl.dtype}; K/V {nbytes / 1e9:.2f} GB > L2",
+            "splits": p.splits, "ms": ms, "GB_per_s": gbs, "peak_GB_per_s": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes,
+            "tokens_per_s": DECODE_BATCH / (ms * 1e-3)}
+
+
 def e2e_steps(inp, dw, steps, stream):
     """End to end through the public API: pinned host inputs -> device, prefill + combine for
     every piece, outputs -> pinned host, every step. Returns (per-step ms, h2d, d2h bytes)."""
@@ -381,6 +436,11 @@ def gpu_arm(args):
     if paged and not args.no_kv_append:
         kv = kv_append_measure(inp, dev, stream, peaks)
 
+    # ---- batched paged decode on a cache of the same shape (its own HBM roofline)
+    dec = None
+    if paged and not args.no_decode:
+        dec = decode_measure(wl, dev, stream, peaks)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e and paged:
@@ -427,6 +487,7 @@ def gpu_arm(args):
                      "algorithmic_flops_per_step": flops},
         "e2e": e2e,
         "kv_append": kv,
+        "decode": dec,
         "cpu_baseline": cpu,
         "gpu_launches": launches,
         "clocks": clocks,
@@ -451,6 +512,7 @@ def main(argv=None):
     ap.add_argument("--l2-flush-mb", type=int, default=L2_FLUSH_BYTES >> 20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-kv-append", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)

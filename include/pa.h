@@ -106,7 +106,7 @@ typedef struct {
   int32_t policy;         /* pa_policy used (or -1 when splits was overridden); balanced
                            * plans read PA_POLICY_BALANCED whichever policy chose them */
   int32_t ctas_per_unit;  /* 2: head_dim 256 runs on CTA pairs (two Q tiles per unit); else 1 */
-  int32_t reserved;
+  int32_t batch;          /* decode plans (pa_decode_plan): sequences; prefill plans: 0 */
   int64_t hist_len;       /* H: keys in the cache before the piece */
   int64_t units;          /* Hkv * ceil(q_tiles / ctas_per_unit) * S units (CTAs or pairs);
                            * balanced: the number of items */
@@ -179,6 +179,39 @@ int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_pool, const v
  */
 int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes, float* out,
                pa_stream_t stream);
+
+/*
+ * pa_decode_plan — plan batched paged decode attention: `batch` sequences, one new query token
+ * each (its own K/V already in the pool), every key of the sequence visible. Fills a plan whose
+ * chunk_rows = batch (one row per sequence), q_tiles = 1 (needs G <= 128), batch = batch and
+ * splits S: the history of every sequence is cut into S splits so that batch * Hkv * S units
+ * fill num_sms SMs (about two per SM, at most 32 and at most the 128-key tiles of
+ * max_seq_len), or exactly splits_override. ws_bytes = S * batch * Hq * (D + 1) * 4 when S > 1,
+ * in the layout of pa_prefill's split workspace with batch in place of R, so pa_combine
+ * merges it. Returns PA_OK, PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED. Pure host code.
+ * Source: the paged decode slowdown the pages measure (decode on the same paged cache).
+ */
+int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_size,
+                   int batch, int64_t max_seq_len, int dtype, float scale, int splits_override,
+                   pa_plan_t* plan);
+
+/*
+ * pa_decode — batched paged decode attention on `stream` (single-CTA kernel at every head dim).
+ *   q            device [batch][Hq][D] of dtype: the new token of each sequence.
+ *   k_pool,v_pool device [num_pages][PS][Hkv][D], 16-byte aligned.
+ *   block_table  device int32 [batch][table_stride]: sequence b's logical page -> physical page.
+ *   seq_lens     device int32 [batch]: keys of sequence b (its new token included), 0..
+ *                table_stride * PS. A sequence with no key gets zeros. A length outside that
+ *                range is clamped into it and reported as PA_ERR_PAGE_INDEX by pa_device_error.
+ *   out          device fp32 [batch][Hq][D]. Written when plan->splits == 1.
+ *   lse_ws       workspace of plan->ws_bytes when S > 1; then call pa_combine (same plan).
+ * Returns PA_OK, PA_ERR_INVALID_ARG, PA_ERR_WORKSPACE or PA_ERR_CUDA; bad page entries and
+ * wait timeouts are reported by pa_device_error.
+ */
+int pa_decode(const pa_plan_t* plan, const void* q, const void* k_pool, const void* v_pool,
+              const int32_t* block_table, int table_stride, const int32_t* seq_lens,
+              int64_t num_pages, float* out, float* lse_ws, uint64_t ws_bytes,
+              pa_stream_t stream);
 
 /* Bytes of the device-resident scratch used by pa_prefill_noalloc (64 MiB). */
 #define PA_NOALLOC_WS_BYTES (64ull << 20)

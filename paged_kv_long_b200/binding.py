@@ -22,7 +22,8 @@ STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "P
 EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_device_error",
             "pa_set_wait_timeout_ns",
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
-            "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append", "pa_pieces")
+            "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append", "pa_pieces",
+            "pa_decode_plan", "pa_decode")
 
 
 class PaError(RuntimeError):
@@ -38,7 +39,8 @@ class Plan(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("group", ctypes.c_int32),
         ("chunk_rows", ctypes.c_int32), ("q_tiles", ctypes.c_int32), ("splits", ctypes.c_int32),
         ("paged", ctypes.c_int32), ("dtype", ctypes.c_int32), ("policy", ctypes.c_int32),
-        ("ctas_per_unit", ctypes.c_int32), ("reserved", ctypes.c_int32), ("hist_len", ctypes.c_int64), ("units", ctypes.c_int64), ("scale", ctypes.c_float),
+        ("ctas_per_unit", ctypes.c_int32), ("batch", ctypes.c_int32), ("hist_len", ctypes.c_int64),
+        ("units", ctypes.c_int64), ("scale", ctypes.c_float),
         ("est_us", ctypes.c_float), ("ws_bytes", ctypes.c_uint64),
     ]
 
@@ -90,6 +92,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_kv_append.restype = i32
     lib.pa_pieces.argtypes = [i32, i64, i32, ctypes.POINTER(ctypes.c_int32), i32]
     lib.pa_pieces.restype = i32
+    lib.pa_decode_plan.argtypes = [i32, i32, i32, i32, i32, i32, i64, i32, ctypes.c_float, i32,
+                                   ctypes.POINTER(Plan)]
+    lib.pa_decode_plan.restype = i32
+    lib.pa_decode.argtypes = [ctypes.POINTER(Plan), vp, vp, vp, vp, i32, vp, i64, vp, vp, u64, vp]
+    lib.pa_decode.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -281,6 +288,57 @@ def prefill_noalloc(p: Plan, q, k_pool, v_pool, page_table, out, stream=None):
                                            v_pool.data_ptr(), tab, num_pages, p.hist_len, R,
                                            out.data_ptr(), _stream_ptr(stream))
     _check(st, "pa_prefill_noalloc")
+
+
+def decode_plan(n_q_heads: int, n_kv_heads: int, head_dim: int, page_size: int, batch: int,
+                max_seq_len: int, dtype="bf16", scale: float = 0.0, splits: int = 0,
+                num_sms: int | None = None) -> Plan:
+    """pa_decode_plan: split count and workspace for one batched decode step (host only)."""
+    if num_sms is None:
+        import torch
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    p = Plan()
+    st = load_library().pa_decode_plan(num_sms, n_q_heads, n_kv_heads, head_dim, page_size, batch,
+                                       max_seq_len, _dtype_code(dtype), scale, splits,
+                                       ctypes.byref(p))
+    _check(st, "pa_decode_plan")
+    return p
+
+
+def decode(p: Plan, q, k_pool, v_pool, block_table, seq_lens, out=None, ws=None, stream=None):
+    """pa_decode followed by pa_combine: one query token per sequence against that sequence's
+    paged keys. q [B, Hq, D]; block_table int32 [B, max_pages]; seq_lens int32 [B] (keys of
+    each sequence, the new token's included). Returns out fp32 [B, Hq, D]."""
+    import torch
+    dt = _torch_dtype(p)
+    B, Hq, Hkv, D, PS = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.page_size
+    _require_cuda(q, "q", dt, (B, Hq, D))
+    _require_cuda(k_pool, "k_pool", dt)
+    _require_cuda(v_pool, "v_pool", dt, tuple(k_pool.shape))
+    if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (PS, Hkv, D):
+        raise ValueError("k_pool must be [num_pages, page_size, Hkv, D]")
+    _require_cuda(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [batch, max_pages]")
+    _require_cuda(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    _require_cuda(out, "out", torch.float32, (B, Hq, D))
+    ws_ptr, ws_bytes = None, 0
+    if p.ws_bytes > 0:
+        if ws is None:
+            ws = workspace(p, q.device)
+        _require_cuda(ws, "ws", torch.float32)
+        ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * 4
+    lib = load_library()
+    st = lib.pa_decode(ctypes.byref(p), q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                       block_table.data_ptr(), block_table.stride(0), seq_lens.data_ptr(),
+                       k_pool.shape[0], out.data_ptr(), ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(st, "pa_decode")
+    if p.ws_bytes > 0:
+        _check(lib.pa_combine(ctypes.byref(p), ws_ptr, ws_bytes, out.data_ptr(),
+                              _stream_ptr(stream)), "pa_combine")
+    return out
 
 
 def device_error(reset: bool = True) -> tuple[int, int]:

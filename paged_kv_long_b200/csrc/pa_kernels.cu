@@ -74,6 +74,13 @@ struct PrefillArgs {
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
   int32_t q_tma;           // 1: the Q tile arrives by tensor copy (CTA-pair kernel, G | 128)
+  int64_t ws_split_rows;   // workspace rows of one split: R * Hq (decode: batch * Hq)
+  // Batched decode (batch > 0, single-CTA kernel): unit u is (sequence u / (Hkv*S), KV head,
+  // split); sequence b has seq_lens[b] keys, its page-table row at page_table + b * table_stride,
+  // its one query token at q + b*Hq*D and its output rows at out + b*Hq*D.
+  int32_t batch;
+  int32_t table_stride;
+  const int32_t* seq_lens;
   int32_t balanced;        // 1: CTA (pair) b runs work item b of the item table
   int32_t rows_per_block;  // packed rows of a row block (balanced workspace slots)
 };
@@ -405,7 +412,7 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       if (x.slot >= 0)
         ws_row = (int64_t)x.slot * a.rows_per_block + x.row0 + r;
       else if (x.slot == kSlotUniform && a.splits > 1)
-        ws_row = ((int64_t)s * a.R + tok) * a.Hq + head;
+        ws_row = (int64_t)s * a.ws_split_rows + tok * a.Hq + head;
       float* dst = ws_row < 0 ? a.out + (tok * a.Hq + head) * (int64_t)D : a.ws_o + ws_row * D;
       // The row goes through shared memory (the K/V ring, idle now; rows 16 bytes apart from
       // a multiple of 128 so a warp's stores spread over the banks) and leaves as one
@@ -444,7 +451,8 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
 template <int D, bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const PrefillArgs a, const __grid_constant__ ItemTable items) {
+                   const PrefillArgs a_in, const __grid_constant__ ItemTable items) {
+  PrefillArgs a = a_in;  // rebased on one sequence in batched decode
   using C = Cfg<D>;
   constexpr int NP = C::NP, NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
@@ -462,6 +470,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     kt0 = it.kt0;
     kt1 = it.kt1;
     slot = it.slot;
+  } else if (a.batch > 0) {
+    // one new token of sequence b: keys 0 .. len-1 (its own included), all visible
+    const int64_t per_seq = (int64_t)a.Hkv * a.splits;
+    const int64_t b = blockIdx.x / per_seq, rem = blockIdx.x % per_seq;
+    g = (int)(rem / a.splits);
+    s = (int)(rem % a.splits);
+    qt = 0;
+    int64_t len = __ldg(a.seq_lens + b);
+    const int64_t cap = (int64_t)a.table_stride * a.page_rows;  // keys the table row can map
+    if (len < 0 || len > cap) {  // reported like a bad page entry; the length is clamped
+      if (threadIdx.x == 0 && g == 0 && s == 0) atomicOr(&g_pa_error_flags, kFlagPage);
+      len = len < 0 ? 0 : cap;
+    }
+    a.q += b * a.Hq * D;
+    a.out += b * a.Hq * D;
+    if (a.ws_o) {
+      a.ws_o += b * a.Hq * D;
+      a.ws_lse += b * a.Hq;
+    }
+    a.page_table += b * a.table_stride;
+    a.hist_len = len > 0 ? len - 1 : 0;
+    a.total_keys = len;
+    a.table_len = (len + a.page_rows - 1) / a.page_rows;
+    a.R = len > 0 ? 1 : 0;
+    split_range((len + kTileKeys - 1) / kTileKeys, s, a.splits, &kt0, &kt1);
   } else {
     unit_coords(blockIdx.x, a.q_tiles, a.Hkv, a.splits, &qt, &g, &s);
     split_range(tile_kv_tiles(qt, a.R, a.G, a.hist_len), s, a.splits, &kt0, &kt1);
@@ -472,12 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x < kTileRows) {
       const int64_t grow = qt * kTileRows + threadIdx.x;
       const int64_t tok = grow / a.G;
-      if (tok < a.R) {
+      if (tok < (a.batch > 0 ? 1 : a.R)) {
         const int head = g * a.G + (int)(grow % a.G);
-        const int64_t row = ((int64_t)s * a.R + tok) * a.Hq + head;
-        float4* d4 = reinterpret_cast<float4*>(a.ws_o + row * D);
-        for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        a.ws_lse[row] = -INFINITY;
+        if (a.splits == 1) {  // decode of a sequence with no key: zeros
+          float4* d4 = reinterpret_cast<float4*>(a.out + (tok * a.Hq + head) * D);
+          for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          const int64_t row = (int64_t)s * a.ws_split_rows + tok * a.Hq + head;
+          float4* d4 = reinterpret_cast<float4*>(a.ws_o + row * D);
+          for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          a.ws_lse[row] = -INFINITY;
+        }
       }
     }
     return;
@@ -993,7 +1031,7 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
                           const void* v_pool, const int32_t* page_table, int64_t num_pages,
                           int64_t hist_len, int chunk_rows, float* out, float* lse_ws,
                           uint64_t ws_bytes, pa_stream_t stream) {
-  if (!plan || !q || !k_pool || !v_pool) return PA_ERR_INVALID_ARG;
+  if (!plan || !q || !k_pool || !v_pool || plan->batch != 0) return PA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool)) return PA_ERR_INVALID_ARG;
   if (hist_len != plan->hist_len || chunk_rows != plan->chunk_rows || chunk_rows <= 0)
     return PA_ERR_INVALID_ARG;
@@ -1076,6 +1114,10 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.scale_log2 = plan->scale * 1.4426950408889634f;
   a.timeout_ns = g_timeout_ns.load();
   a.balanced = balanced ? 1 : 0;
+  a.ws_split_rows = (int64_t)chunk_rows * plan->n_q_heads;
+  a.batch = 0;
+  a.table_stride = 0;
+  a.seq_lens = nullptr;
   a.q_tma = q_tma ? 1 : 0;
   a.rows_per_block = per * kTileRows;
   // Kernel parameter of 8 KB, copied into the launch: kept off the stack of callers with small
@@ -1095,6 +1137,76 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
                 : (bf16 ? launch_pair<false, true>(grid, st, tk, tv, tq, a, *tab)
                         : launch_pair<false, false>(grid, st, tk, tv, tq, a, *tab));
       break;
+  }
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_decode(const pa_plan_t* plan, const void* q, const void* k_pool,
+                         const void* v_pool, const int32_t* block_table, int table_stride,
+                         const int32_t* seq_lens, int64_t num_pages, float* out, float* lse_ws,
+                         uint64_t ws_bytes, pa_stream_t stream) {
+  if (!plan || plan->batch <= 0 || plan->chunk_rows != plan->batch || plan->q_tiles != 1)
+    return PA_ERR_INVALID_ARG;
+  if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !out || table_stride <= 0 ||
+      num_pages <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  const int D = plan->head_dim, S = plan->splits, B = plan->batch, PS = plan->page_size;
+  if (D != 64 && D != 128 && D != 256) return PA_ERR_UNSUPPORTED;
+  if (S < 1 || S > PA_MAX_SPLITS || plan->n_q_heads != plan->n_kv_heads * plan->group ||
+      plan->group > kTileRows || plan->units != (int64_t)B * plan->n_kv_heads * S)
+    return PA_ERR_INVALID_ARG;
+  if (S > 1 && (!lse_ws || !aligned16(lse_ws) || ws_bytes < plan->ws_bytes))
+    return PA_ERR_WORKSPACE;
+  if (num_pages * PS + kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  const bool bf16 = plan->dtype == PA_BF16;
+  const int64_t rows = num_pages * PS;
+  const int v_rows = std::min(PS, 128 / (D / 64));
+  CUtensorMap tk, tv;
+  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, PS) ||
+      !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, D / 64))
+    return PA_ERR_CUDA;
+  PrefillArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = static_cast<const uint16_t*>(q);
+  a.page_table = block_table;
+  a.out = out;
+  a.ws_o = S > 1 ? lse_ws : nullptr;
+  a.ws_lse = S > 1 ? lse_ws + (int64_t)S * B * plan->n_q_heads * D : nullptr;
+  a.R = 1;
+  a.Hq = plan->n_q_heads;
+  a.Hkv = plan->n_kv_heads;
+  a.G = plan->group;
+  a.q_tiles = 1;
+  a.splits = S;
+  a.page_rows = PS;
+  a.page_shift = __builtin_ctz((unsigned)PS);
+  a.pages_per_tile = kTileKeys / PS;
+  a.k_rows = PS;
+  a.v_rows = v_rows;
+  a.v_shift = __builtin_ctz((unsigned)v_rows);
+  a.num_pages = (int32_t)num_pages;
+  a.oob_row = (int32_t)rows;
+  a.scale_log2 = plan->scale * 1.4426950408889634f;
+  a.timeout_ns = g_timeout_ns.load();
+  a.rows_per_block = kTileRows;
+  a.ws_split_rows = (int64_t)B * plan->n_q_heads;
+  a.batch = B;
+  a.table_stride = table_stride;
+  a.seq_lens = seq_lens;
+  thread_local ItemTable table;  // unused by decode units
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t grid = plan->units;
+  if (grid >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  cudaError_t e;
+  switch (D) {
+    case 64: e = bf16 ? launch_prefill<64, true, true>(grid, st, tk, tv, a, table)
+                      : launch_prefill<64, true, false>(grid, st, tk, tv, a, table); break;
+    case 128: e = bf16 ? launch_prefill<128, true, true>(grid, st, tk, tv, a, table)
+                       : launch_prefill<128, true, false>(grid, st, tk, tv, a, table); break;
+    default: e = bf16 ? launch_prefill<256, true, true>(grid, st, tk, tv, a, table)
+                      : launch_prefill<256, true, false>(grid, st, tk, tv, a, table); break;
   }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

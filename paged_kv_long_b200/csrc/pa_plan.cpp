@@ -204,6 +204,53 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
 
 }  // namespace pa
 
+extern "C" int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
+                              int page_size, int batch, int64_t max_seq_len, int dtype,
+                              float scale, int splits_override, pa_plan_t* plan) {
+  if (!plan) return PA_ERR_INVALID_ARG;
+  memset(plan, 0, sizeof *plan);
+  if (num_sms <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || batch <= 0 || max_seq_len < 1)
+    return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (splits_override < 0 || !(scale >= 0.0f) || isinf(scale)) return PA_ERR_INVALID_ARG;
+  if (n_q_heads % n_kv_heads) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (!is_pow2(page_size) || page_size < 16 || page_size > 128) return PA_ERR_UNSUPPORTED;
+  if (splits_override > PA_MAX_SPLITS) return PA_ERR_UNSUPPORTED;
+  const int G = n_q_heads / n_kv_heads;
+  if (G > pa::kTileRows) return PA_ERR_UNSUPPORTED;
+  if (max_seq_len + pa::kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  const int64_t max_tiles = pa::ceil_div64(max_seq_len, pa::kTileKeys);
+  int S = splits_override;
+  if (S == 0) {  // about two units per SM
+    const int64_t want = pa::ceil_div64(2LL * num_sms, (int64_t)batch * n_kv_heads);
+    S = (int)std::max<int64_t>(1, std::min<int64_t>({want, (int64_t)PA_MAX_SPLITS, max_tiles}));
+  }
+  if ((int64_t)batch * n_kv_heads * S >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  const CostModel cm(head_dim);
+  plan->num_sms = num_sms;
+  plan->n_q_heads = n_q_heads;
+  plan->n_kv_heads = n_kv_heads;
+  plan->head_dim = head_dim;
+  plan->page_size = page_size;
+  plan->group = G;
+  plan->chunk_rows = batch;
+  plan->q_tiles = 1;
+  plan->splits = S;
+  plan->paged = 1;
+  plan->dtype = dtype;
+  plan->policy = splits_override > 0 ? -1 : PA_POLICY_MAKESPAN;
+  plan->ctas_per_unit = 1;
+  plan->batch = batch;
+  plan->hist_len = max_seq_len;
+  plan->units = (int64_t)batch * n_kv_heads * S;
+  plan->scale = scale > 0.0f ? scale : (float)(1.0 / sqrt((double)head_dim));
+  const double waves = std::ceil((double)plan->units / num_sms);
+  plan->est_us = (float)(waves * (cm.unit_us + (double)max_tiles / S * cm.tile_us));
+  plan->ws_bytes = S > 1 ? (uint64_t)S * batch * n_q_heads * (head_dim + 1) * 4ull : 0ull;
+  return PA_OK;
+}
+
 extern "C" int pa_pieces(int chunk_rows, int64_t hist_len, int log2_budget, int32_t* rows_out,
                          int cap) {
   if (chunk_rows < 0 || hist_len < 0 || log2_budget < 1 || log2_budget > 62 || cap < 0)
@@ -298,7 +345,7 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
   plan->dtype = dtype;
   plan->policy = used_policy;
   plan->ctas_per_unit = per;
-  plan->reserved = 0;
+  plan->batch = 0;
   plan->hist_len = hist_len;
   plan->units = q_units * n_kv_heads * S;
   plan->scale = scale > 0.0f ? scale : (float)(1.0 / sqrt((double)head_dim));

@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tok = grow / a.G;
       if (tok < a.R) {
         const int head = g * a.G + (int)(grow % a.G);
-        const int64_t row = ((int64_t)s * a.R + tok) * a.Hq + head;
+        const int64_t row = (int64_t)s * a.ws_split_rows + tok * a.Hq + head;
         float4* d4 = reinterpret_cast<float4*>(a.ws_o + row * D);
         for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         a.ws_lse[row] = -INFINITY;

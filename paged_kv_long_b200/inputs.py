@@ -192,3 +192,61 @@ def small_problem(seed: int, R: int, H: int, Hq: int, Hkv: int, D: int, PS: int,
     k_pool = scatter_to_pool(k, table, pool_pages, PS, fill)
     v_pool = scatter_to_pool(v, table, pool_pages, PS, fill)
     return q, k_pool, v_pool, table, k, v
+
+
+@dataclass
+class DecodeBatch:
+    """One batched decode step over a shared page pool (host side, 16-bit patterns / int32).
+
+    Sequence b holds seq_lens[b] keys (its new token's included) on the pages
+    block_table[b, :ceil(seq_lens[b]/PS)]; its one query token is q[b]. The pages of different
+    sequences are disjoint; table entries past a sequence's pages are -1, and pool slots that
+    no sequence owns hold NaN, so neither may reach an output.
+    """
+    q: np.ndarray            # [B, Hq, D]
+    k_pool: np.ndarray       # [pool_pages, PS, Hkv, D]
+    v_pool: np.ndarray
+    block_table: np.ndarray  # int32 [B, max_pages]
+    seq_lens: np.ndarray     # int32 [B]
+    dtype: str
+    scale: float = 0.0
+
+
+def decode_batch(seed: int, seq_lens, Hq: int, Hkv: int, D: int, PS: int, dtype: str,
+                 pool_factor: float = 1.1, poison: bool = True) -> DecodeBatch:
+    """Seeded N(0, 1) Q/K/V for a batch of sequences of the given key counts; the pages of all
+    sequences are drawn from one shuffled pool."""
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    B = len(lens)
+    pages = [max(0, math.ceil(int(n) / PS)) for n in lens]
+    need = sum(pages)
+    pool_pages = max(1, math.ceil(need * pool_factor))
+    max_pages = max(1, max(pages))
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(pool_pages).astype(np.int32)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    fill = NAN_BITS[dtype] if poison else 0
+    k_pool = np.full((pool_pages, PS, Hkv, D), fill, dtype=np.uint16)
+    v_pool = np.full((pool_pages, PS, Hkv, D), fill, dtype=np.uint16)
+    q = to_bits(rng.standard_normal((B, Hq, D), dtype=np.float32), dtype)
+    at = 0
+    for b in range(B):
+        n, p = int(lens[b]), pages[b]
+        table[b, :p] = perm[at:at + p]
+        at += p
+        if n:
+            k = to_bits(rng.standard_normal((n, Hkv, D), dtype=np.float32), dtype)
+            v = to_bits(rng.standard_normal((n, Hkv, D), dtype=np.float32), dtype)
+            _place(k_pool, k, table[b, :p], PS)
+            _place(v_pool, v, table[b, :p], PS)
+    return DecodeBatch(q, k_pool, v_pool, table, lens.astype(np.int32), dtype)
+
+
+def _place(pool: np.ndarray, logical: np.ndarray, pages: np.ndarray, PS: int):
+    """Write logical rows [n, Hkv, D] into the pool pages listed in order (in place)."""
+    n = logical.shape[0]
+    full = n // PS
+    if full:
+        pool[pages[:full]] = logical[:full * PS].reshape(full, PS, *logical.shape[1:])
+    if n - full * PS:
+        pool[pages[full], :n - full * PS] = logical[full * PS:]
