@@ -297,19 +297,30 @@ def decode_measure(wl, dev, stream, peaks, reps=20, seed=6000):
     out = torch.empty((DECODE_BATCH, wl.n_q_heads, wl.head_dim), dtype=torch.float32,
                       device=dev)
     ws = binding.workspace(p, dev)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            binding.decode(p, q, kp, vp, tab, sl, out, ws, stream)
-        evs = []
-        for _ in range(reps):
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            binding.decode(p, q, kp, vp, tab, sl, out, ws, stream)
-            e1.record(stream)
-            evs.append((e0, e1))
-        torch.cuda.synchronize()
-    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    # the same step as a batch of one-row chunks: host lengths, balanced items
+    bp = binding.batch_plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.page_size,
+                            np.ones(DECODE_BATCH, dtype=np.int32), lens - 1, wl.dtype)
+    ws_b = binding.workspace(bp.plan, dev)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            evs = []
+            for _ in range(reps):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                evs.append((e0, e1))
+            torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+    ms = timed(lambda: binding.decode(p, q, kp, vp, tab, sl, out, ws, stream))
+    ms_b = timed(lambda: binding.batch_prefill(bp, q.view(DECODE_BATCH, wl.n_q_heads,
+                                                          wl.head_dim), kp, vp, tab, out, ws_b,
+                                               stream))
     keys = int(lens.sum())
     nbytes = (2 * keys * wl.n_kv_heads * wl.head_dim * 2            # K and V rows
               + DECODE_BATCH * wl.n_q_heads * wl.head_dim * (2 + 4))  # Q in, fp32 out
@@ -320,7 +331,11 @@ def decode_measure(wl, dev, stream, peaks, reps=20, seed=6000):
                         f"{wl.dtype}; K/V {nbytes / 1e9:.2f} GB > L2",
             "splits": p.splits, "ms": ms, "GB_per_s": gbs, "peak_GB_per_s": peaks["hbm_gbs"],
             "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes,
-            "tokens_per_s": DECODE_BATCH / (ms * 1e-3)}
+            "tokens_per_s": DECODE_BATCH / (ms * 1e-3),
+            "balanced": {"how": "pa_batch_prefill with one row per sequence (host lengths)",
+                         "items": int(bp.plan.units), "ms": ms_b,
+                         "GB_per_s": nbytes / (ms_b * 1e-3) / 1e9,
+                         "frac": nbytes / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
 
 
 def e2e_steps(inp, dw, steps, stream):

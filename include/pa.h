@@ -213,6 +213,57 @@ int pa_decode(const pa_plan_t* plan, const void* q, const void* k_pool, const vo
               int64_t num_pages, float* out, float* lse_ws, uint64_t ws_bytes,
               pa_stream_t stream);
 
+/*
+ * Batched prefill (continuous batching): several sequences in one launch, each a chunk of
+ * q_lens[b] query rows at its own history of hist_lens[b] keys, all on one page pool. The
+ * causal rule is the single-piece one, per sequence: row i of sequence b sees keys
+ * 0 .. hist_lens[b] + i of that sequence. A decode step is the case q_lens[b] = 1,
+ * hist_lens[b] = keys before the new token. Source: the pages' chunked prefill (BaseRT issue
+ * #51, "Results"; splash PR #33, "What changed") applied to every sequence of a batch; the
+ * batching itself is the serving engine's, which the pages do not describe.
+ *
+ * pa_batch_plan — the balanced schedule of the batch (host only): the row blocks of all
+ * sequences, longest first, cut by the wrap-around rule into at most 512 items on num_sms SMs.
+ *   q_lens     host int32 [batch], >= 0 (a sequence with 0 rows has no output rows).
+ *   hist_lens  host int64 [batch], >= 0.
+ *   batch      1 .. 256 sequences; at most 512 row blocks in all ((KV head, 128-row Q tile
+ *              unit) pairs: Hkv * ceil(ceil(q_lens[b] * G / 128) / ctas_per_unit) summed).
+ * Fills a plan with batch = batch, chunk_rows = sum of q_lens, hist_len = the largest history,
+ * policy = PA_POLICY_BALANCED, units = items, splits = the most items of one row block, and
+ * ws_bytes = slots * ctas_per_unit*128 * (D + 1) * 4. The arrays are not kept: pass the same
+ * ones to pa_batch_prefill and pa_batch_combine, which rebuild the schedule from them.
+ * Returns PA_OK, PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED (too many sequences or row blocks).
+ */
+int pa_batch_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_size,
+                  int batch, const int32_t* q_lens, const int64_t* hist_lens, int dtype,
+                  float scale, pa_plan_t* plan);
+
+/*
+ * pa_batch_prefill — batched prefill attention on `stream`.
+ *   q            device [sum q_lens][Hq][D] of dtype: the sequences' chunks, packed in order.
+ *   k_pool,v_pool device [num_pages][PS][Hkv][D]; the chunks' own K/V already in place.
+ *   block_table  device int32 [batch][table_stride]: sequence b's logical page -> physical page;
+ *                entries past ceil((hist_lens[b] + q_lens[b]) / PS) are not read.
+ *   out          device fp32 [sum q_lens][Hq][D]; rows of uncut row blocks are written here.
+ *   lse_ws       workspace of plan->ws_bytes when ws_bytes > 0; then call pa_batch_combine.
+ * Returns PA_OK, PA_ERR_INVALID_ARG (arrays that do not rebuild the plan's schedule, or a
+ * plan that is not a batch plan), PA_ERR_WORKSPACE or PA_ERR_CUDA.
+ */
+int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens, const int64_t* hist_lens,
+                     const void* q, const void* k_pool, const void* v_pool,
+                     const int32_t* block_table, int table_stride, int64_t num_pages, float* out,
+                     float* lse_ws, uint64_t ws_bytes, pa_stream_t stream);
+
+/* pa_batch_schedule_items — the work items of a batch plan, as pa_schedule_items lists them;
+ * rb is a global row block: sequence b owns rb0_b .. rb0_b + its row blocks - 1, with rb0_b
+ * the row blocks of sequences 0 .. b-1, numbered within the sequence like a single piece's. */
+int pa_batch_schedule_items(const pa_plan_t* plan, const int32_t* q_lens,
+                            const int64_t* hist_lens, int32_t* items, int cap);
+
+/* pa_batch_combine — merge the partials of the cut row blocks into out (no-op when none). */
+int pa_batch_combine(const pa_plan_t* plan, const int32_t* q_lens, const int64_t* hist_lens,
+                     const float* lse_ws, uint64_t ws_bytes, float* out, pa_stream_t stream);
+
 /* Bytes of the device-resident scratch used by pa_prefill_noalloc (64 MiB). */
 #define PA_NOALLOC_WS_BYTES (64ull << 20)
 

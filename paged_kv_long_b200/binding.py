@@ -23,7 +23,8 @@ EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_dev
             "pa_set_wait_timeout_ns",
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
             "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append", "pa_pieces",
-            "pa_decode_plan", "pa_decode")
+            "pa_decode_plan", "pa_decode", "pa_batch_plan", "pa_batch_prefill",
+            "pa_batch_combine", "pa_batch_schedule_items")
 
 
 class PaError(RuntimeError):
@@ -97,6 +98,17 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_decode_plan.restype = i32
     lib.pa_decode.argtypes = [ctypes.POINTER(Plan), vp, vp, vp, vp, i32, vp, i64, vp, vp, u64, vp]
     lib.pa_decode.restype = i32
+    lib.pa_batch_plan.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, i32, ctypes.c_float,
+                                  ctypes.POINTER(Plan)]
+    lib.pa_batch_plan.restype = i32
+    lib.pa_batch_prefill.argtypes = [ctypes.POINTER(Plan), vp, vp, vp, vp, vp, vp, i32, i64, vp,
+                                     vp, u64, vp]
+    lib.pa_batch_prefill.restype = i32
+    lib.pa_batch_combine.argtypes = [ctypes.POINTER(Plan), vp, vp, vp, u64, vp, vp]
+    lib.pa_batch_combine.restype = i32
+    lib.pa_batch_schedule_items.argtypes = [ctypes.POINTER(Plan), vp, vp,
+                                            ctypes.POINTER(ctypes.c_int32), i32]
+    lib.pa_batch_schedule_items.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -338,6 +350,91 @@ def decode(p: Plan, q, k_pool, v_pool, block_table, seq_lens, out=None, ws=None,
     if p.ws_bytes > 0:
         _check(lib.pa_combine(ctypes.byref(p), ws_ptr, ws_bytes, out.data_ptr(),
                               _stream_ptr(stream)), "pa_combine")
+    return out
+
+
+class BatchPlan:
+    """A batched plan with the host length arrays it was made from (pa_batch_plan)."""
+
+    def __init__(self, plan: Plan, q_lens, hist_lens):
+        import numpy as np
+        self.plan = plan
+        self.q_lens = np.ascontiguousarray(q_lens, dtype=np.int32)
+        self.hist_lens = np.ascontiguousarray(hist_lens, dtype=np.int64)
+
+    def _arrays(self):
+        return self.q_lens.ctypes.data, self.hist_lens.ctypes.data
+
+
+def batch_plan(n_q_heads: int, n_kv_heads: int, head_dim: int, page_size: int, q_lens,
+               hist_lens, dtype="bf16", scale: float = 0.0,
+               num_sms: int | None = None) -> BatchPlan:
+    """pa_batch_plan: the balanced schedule of a batch of chunks (host only)."""
+    import numpy as np
+    if num_sms is None:
+        import torch
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    q_lens = np.ascontiguousarray(q_lens, dtype=np.int32)
+    hist_lens = np.ascontiguousarray(hist_lens, dtype=np.int64)
+    if q_lens.shape != hist_lens.shape or q_lens.ndim != 1:
+        raise ValueError("q_lens and hist_lens must be 1-D of the same length")
+    p = Plan()
+    st = load_library().pa_batch_plan(num_sms, n_q_heads, n_kv_heads, head_dim, page_size,
+                                      len(q_lens), q_lens.ctypes.data, hist_lens.ctypes.data,
+                                      _dtype_code(dtype), scale, ctypes.byref(p))
+    _check(st, "pa_batch_plan")
+    return BatchPlan(p, q_lens, hist_lens)
+
+
+def batch_schedule_items(bp: BatchPlan):
+    """pa_batch_schedule_items: int32 [n, 4] of (global row block, kt0, kt1, slot or -1)."""
+    import numpy as np
+    lib = load_library()
+    ql, hl = bp._arrays()
+    n = lib.pa_batch_schedule_items(ctypes.byref(bp.plan), ql, hl, None, 0)
+    if n < 0:
+        raise PaError(n, "pa_batch_schedule_items")
+    out = np.zeros((max(n, 1), 4), dtype=np.int32)
+    lib.pa_batch_schedule_items(ctypes.byref(bp.plan), ql, hl,
+                                out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n)
+    return out[:n]
+
+
+def batch_prefill(bp: BatchPlan, q, k_pool, v_pool, block_table, out=None, ws=None,
+                  stream=None):
+    """pa_batch_prefill followed by pa_batch_combine. q [sum q_lens, Hq, D] (the sequences'
+    chunks packed in order); block_table int32 [batch, max_pages]. Returns out fp32
+    [sum q_lens, Hq, D]."""
+    import torch
+    p = bp.plan
+    dt = _torch_dtype(p)
+    rows, Hq, Hkv, D, PS = p.chunk_rows, p.n_q_heads, p.n_kv_heads, p.head_dim, p.page_size
+    _require_cuda(q, "q", dt, (rows, Hq, D))
+    _require_cuda(k_pool, "k_pool", dt)
+    _require_cuda(v_pool, "v_pool", dt, tuple(k_pool.shape))
+    if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (PS, Hkv, D):
+        raise ValueError("k_pool must be [num_pages, page_size, Hkv, D]")
+    _require_cuda(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != p.batch:
+        raise ValueError("block_table must be [batch, max_pages]")
+    if out is None:
+        out = torch.empty((rows, Hq, D), dtype=torch.float32, device=q.device)
+    _require_cuda(out, "out", torch.float32, (rows, Hq, D))
+    ws_ptr, ws_bytes = None, 0
+    if p.ws_bytes > 0:
+        if ws is None:
+            ws = workspace(p, q.device)
+        _require_cuda(ws, "ws", torch.float32)
+        ws_ptr, ws_bytes = ws.data_ptr(), ws.numel() * 4
+    ql, hl = bp._arrays()
+    lib = load_library()
+    st = lib.pa_batch_prefill(ctypes.byref(p), ql, hl, q.data_ptr(), k_pool.data_ptr(),
+                              v_pool.data_ptr(), block_table.data_ptr(), block_table.stride(0),
+                              k_pool.shape[0], out.data_ptr(), ws_ptr, ws_bytes,
+                              _stream_ptr(stream))
+    _check(st, "pa_batch_prefill")
+    _check(lib.pa_batch_combine(ctypes.byref(p), ql, hl, ws_ptr, ws_bytes, out.data_ptr(),
+                                _stream_ptr(stream)), "pa_batch_combine")
     return out
 
 

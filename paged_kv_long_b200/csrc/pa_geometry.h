@@ -81,6 +81,27 @@ struct PaSplitBlock {
 constexpr int kMaxItems = 512;
 constexpr int kMaxSplitBlocks = 256;
 
+// ---- batched plans (several sequences, each a chunk of `rows` query rows at its own history)
+//
+// Sequence b owns query/output rows [q_row0, q_row0 + rows) of the packed [sum rows][Hq][D]
+// arrays, has `hist` keys before its chunk, and its row blocks are the global row blocks
+// [rb0, rb0 + its row-block count), numbered within the sequence as above (longest first).
+struct PaSeq {
+  int32_t q_row0, rows, hist, rb0;
+};
+constexpr int kMaxSeqs = 256;
+
+// The sequence that owns global row block rb: the last b with seq[b].rb0 <= rb (rb0 ascending).
+PA_HD int seq_of_rb(const PaSeq* seq, int n, int32_t rb) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (seq[mid].rb0 <= rb) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 PA_HD void rb_coords(int32_t rb, int64_t q_units, int Hkv, int64_t* qu, int* g) {
   *qu = q_units - 1 - rb / Hkv;
   *g = rb % Hkv;

@@ -83,15 +83,39 @@ struct PrefillArgs {
   const int32_t* seq_lens;
   int32_t balanced;        // 1: CTA (pair) b runs work item b of the item table
   int32_t rows_per_block;  // packed rows of a row block (balanced workspace slots)
+  // Batched prefill (balanced and batch > 0): an item's row block names its sequence (the item
+  // table's sequence list); q_row0 is that sequence's first row in the packed Q / out arrays.
+  int32_t q_row0;
 };
+
 
 // The work items of a balanced plan, passed by value (kernel parameter space): no device
 // allocation, and a CUDA graph that captures the launch keeps its own copy.
 struct ItemTable {
   PaItem item[kMaxItems];
+  PaSeq seq[kMaxSeqs];  // batched plans: the sequences, rb0 ascending
 };
 // SoftmaxCtx::slot value of the uniform-split schedule (destination from the split index).
 constexpr int kSlotUniform = -2;
+
+// Batched plans: point the arguments at the sequence that owns global row block rb (its Q and
+// output rows, its page-table row, its history and rows) and return the row block's number
+// within the sequence.
+template <int D>
+__device__ __forceinline__ int32_t batch_rebase(PrefillArgs& a, const ItemTable& t, int32_t rb) {
+  const int b = seq_of_rb(t.seq, a.batch, rb);
+  const PaSeq sq = t.seq[b];
+  a.q += (int64_t)sq.q_row0 * a.Hq * D;
+  a.out += (int64_t)sq.q_row0 * a.Hq * D;
+  a.page_table += (int64_t)b * a.table_stride;
+  a.hist_len = sq.hist;
+  a.R = sq.rows;
+  a.total_keys = (int64_t)sq.hist + sq.rows;
+  a.table_len = (a.total_keys + a.page_rows - 1) / a.page_rows;
+  a.q_tiles = (int32_t)q_tiles_for(sq.rows, a.G);
+  a.q_row0 = sq.q_row0;
+  return rb - sq.rb0;
+}
 
 // Shared-memory layout. The ring holds 16 KB slots, filled and consumed in the order K0, K1,
 // V0, K2, V1, ..., V_{n-1}; every K or V tile takes NP consecutive slots (mod NSLOT). A K
@@ -452,7 +476,7 @@ template <int D, bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const PrefillArgs a_in, const __grid_constant__ ItemTable items) {
-  PrefillArgs a = a_in;  // rebased on one sequence in batched decode
+  PrefillArgs a = a_in;  // rebased on one sequence in batched plans and decode
   using C = Cfg<D>;
   constexpr int NP = C::NP, NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
@@ -465,7 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int g, s, slot = kSlotUniform;
   if (a.balanced) {
     const PaItem it = items.item[blockIdx.x];
-    rb_coords(it.rb, a.q_tiles, a.Hkv, &qt, &g);
+    const int32_t rb = a.batch > 0 ? batch_rebase<D>(a, items, it.rb) : it.rb;
+    rb_coords(rb, a.q_tiles, a.Hkv, &qt, &g);
     s = 0;
     kt0 = it.kt0;
     kt1 = it.kt1;
@@ -823,22 +848,32 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 // Balanced plans: one warp per packed row of a cut row block merges that row's parts (workspace
 // slots first_slot .. first_slot + nparts - 1, at most 32) into out, with the same weighting.
+// Batched plans: the sequences (n_seq > 0), whose row blocks the split blocks name.
 struct SplitTable {
   PaSplitBlock blk[kMaxSplitBlocks];
+  PaSeq seq[kMaxSeqs];
 };
 
 __global__ void __launch_bounds__(256) combine_blocks_kernel(
     const float* __restrict__ ws_o, const float* __restrict__ ws_lse, float* __restrict__ out,
     const __grid_constant__ SplitTable t, int n_blocks, int rows_per_block, int64_t q_units,
-    int Hkv, int G, int R, int Hq, int D) {
+    int Hkv, int G, int R, int Hq, int D, int n_seq) {
   const int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (w >= (int64_t)n_blocks * rows_per_block) return;
   const int lane = threadIdx.x & 31;
   const PaSplitBlock b = t.blk[w / rows_per_block];
   const int lr = (int)(w % rows_per_block);
+  int32_t rb = b.rb;
+  if (n_seq > 0) {  // the owning sequence: its rows, its Q-tile units, its output rows
+    const PaSeq sq = t.seq[seq_of_rb(t.seq, n_seq, rb)];
+    rb -= sq.rb0;
+    R = sq.rows;
+    q_units = ceil_div64(q_tiles_for(sq.rows, G), rows_per_block / kTileRows);
+    out += (int64_t)sq.q_row0 * Hq * D;
+  }
   int64_t qu;
   int g;
-  rb_coords(b.rb, q_units, Hkv, &qu, &g);
+  rb_coords(rb, q_units, Hkv, &qu, &g);
   const int64_t grow = qu * rows_per_block + lr;
   const int64_t tok = grow / G;
   if (tok >= R) return;
@@ -1087,6 +1122,7 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   if (!q_tma) memset(&tq, 0, sizeof tq);
 
   PrefillArgs a;
+  memset(&a, 0, sizeof a);
   a.q = static_cast<const uint16_t*>(q);
   a.page_table = page_table;
   a.out = out;
@@ -1213,7 +1249,8 @@ extern "C" int pa_decode(const pa_plan_t* plan, const void* q, const void* k_poo
 
 extern "C" int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes,
                           float* out, pa_stream_t stream) {
-  if (!plan) return PA_ERR_INVALID_ARG;
+  if (!plan || (plan->policy == PA_POLICY_BALANCED && plan->batch != 0))
+    return PA_ERR_INVALID_ARG;  // batched plans merge with pa_batch_combine
   const int S = plan->splits;
   if (plan->policy == PA_POLICY_BALANCED) {
     Schedule sch;
@@ -1233,7 +1270,7 @@ extern "C" int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t w
                             reinterpret_cast<cudaStream_t>(stream)>>>(
         lse_ws, lse_ws + (int64_t)sch.n_slots * sch.rows_per_block * D, out, table,
         (int)sch.split.size(), sch.rows_per_block, q_units, plan->n_kv_heads, plan->group,
-        plan->chunk_rows, plan->n_q_heads, D);
+        plan->chunk_rows, plan->n_q_heads, D, 0);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
   if (S == 1) return PA_OK;
@@ -1247,6 +1284,128 @@ extern "C" int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t w
   const int64_t blocks = (RH + 7) / 8;
   combine_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       ws_o, ws_lse, out, S, RH, D);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- batched prefill
+namespace pa {
+// The batch and its schedule, rebuilt from the caller's lengths and checked against the plan.
+static int rebuild_batch(const pa_plan_t* plan, const int32_t* q_lens, const int64_t* hist_lens,
+                         Batch* bt, Schedule* sch) {
+  if (!plan || plan->batch <= 0 || plan->policy != PA_POLICY_BALANCED) return PA_ERR_INVALID_ARG;
+  const int D = plan->head_dim;
+  if (D != 64 && D != 128 && D != 256) return PA_ERR_UNSUPPORTED;
+  if (plan->n_kv_heads <= 0 || plan->n_q_heads != plan->n_kv_heads * plan->group ||
+      plan->ctas_per_unit != (D == 256 ? 2 : 1))
+    return PA_ERR_INVALID_ARG;
+  const int st = describe_batch(plan->batch, q_lens, hist_lens, plan->group, plan->n_kv_heads,
+                                plan->ctas_per_unit, bt);
+  if (st != PA_OK) return st;
+  if (!build_batch(plan->num_sms, D, plan->group, plan->n_kv_heads, *bt, sch) ||
+      (int64_t)sch->items.size() != plan->units || bt->total_rows != plan->chunk_rows ||
+      (uint64_t)sch->n_slots * sch->rows_per_block * (D + 1) * 4ull != plan->ws_bytes)
+    return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+}  // namespace pa
+
+extern "C" int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens,
+                                const int64_t* hist_lens, const void* q, const void* k_pool,
+                                const void* v_pool, const int32_t* block_table, int table_stride,
+                                int64_t num_pages, float* out, float* lse_ws, uint64_t ws_bytes,
+                                pa_stream_t stream) {
+  Batch bt;
+  Schedule sch;
+  const int st = rebuild_batch(plan, q_lens, hist_lens, &bt, &sch);
+  if (st != PA_OK) return st;
+  if (!q || !k_pool || !v_pool || !block_table || !out || table_stride <= 0 || num_pages <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  for (const PaSeq& sq : bt.seq)  // every sequence's pages fit its table row
+    if (ceil_div64((int64_t)sq.hist + sq.rows, plan->page_size) > table_stride)
+      return PA_ERR_INVALID_ARG;
+  if (sch.n_slots > 0 && (!lse_ws || !aligned16(lse_ws) || ws_bytes < plan->ws_bytes))
+    return PA_ERR_WORKSPACE;
+  const int D = plan->head_dim, PS = plan->page_size, per = plan->ctas_per_unit;
+  if (num_pages * PS + kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  const bool bf16 = plan->dtype == PA_BF16;
+  const int64_t rows = num_pages * PS;
+  const int k_rows = per == 2 ? std::min(PS, 64) : PS;
+  const int v_rows = per == 2 ? std::min(PS, 64) : std::min(PS, 128 / (D / 64));
+  const int v_panels = per == 2 ? 2 : D / 64;
+  CUtensorMap tk, tv, tq;
+  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows) ||
+      !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, v_panels))
+    return PA_ERR_CUDA;
+  const bool q_tma = per == 2 && kTileRows % plan->group == 0;
+  if (q_tma && !make_q_map(&tq, q, bf16, D, plan->group, plan->n_kv_heads, (int)bt.total_rows))
+    return PA_ERR_CUDA;
+  if (!q_tma) memset(&tq, 0, sizeof tq);
+
+  PrefillArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = static_cast<const uint16_t*>(q);
+  a.page_table = block_table;
+  a.out = out;
+  a.ws_o = sch.n_slots > 0 ? lse_ws : nullptr;
+  a.ws_lse = sch.n_slots > 0 ? lse_ws + (int64_t)sch.n_slots * sch.rows_per_block * D : nullptr;
+  a.Hq = plan->n_q_heads;
+  a.Hkv = plan->n_kv_heads;
+  a.G = plan->group;
+  a.splits = 1;
+  a.page_rows = PS;
+  a.page_shift = __builtin_ctz((unsigned)PS);
+  a.pages_per_tile = kTileKeys / PS;
+  a.k_rows = k_rows;
+  a.v_rows = v_rows;
+  a.v_shift = __builtin_ctz((unsigned)v_rows);
+  a.num_pages = (int32_t)num_pages;
+  a.oob_row = (int32_t)rows;
+  a.scale_log2 = plan->scale * 1.4426950408889634f;
+  a.timeout_ns = g_timeout_ns.load();
+  a.balanced = 1;
+  a.rows_per_block = per * kTileRows;
+  a.q_tma = q_tma ? 1 : 0;
+  a.batch = plan->batch;
+  a.table_stride = table_stride;
+  thread_local ItemTable table;
+  for (size_t i = 0; i < sch.items.size(); ++i) table.item[i] = sch.items[i];
+  for (size_t i = 0; i < bt.seq.size(); ++i) table.seq[i] = bt.seq[i];
+  const int64_t grid = plan->units * per;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  switch (D) {
+    case 64: e = launch_d<64>(true, bf16, grid, cs, tk, tv, a, table); break;
+    case 128: e = launch_d<128>(true, bf16, grid, cs, tk, tv, a, table); break;
+    default:
+      e = bf16 ? launch_pair<true, true>(grid, cs, tk, tv, tq, a, table)
+               : launch_pair<true, false>(grid, cs, tk, tv, tq, a, table);
+      break;
+  }
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_batch_combine(const pa_plan_t* plan, const int32_t* q_lens,
+                                const int64_t* hist_lens, const float* lse_ws, uint64_t ws_bytes,
+                                float* out, pa_stream_t stream) {
+  Batch bt;
+  Schedule sch;
+  const int st = rebuild_batch(plan, q_lens, hist_lens, &bt, &sch);
+  if (st != PA_OK) return st;
+  if (sch.split.empty()) return PA_OK;
+  if (!lse_ws || ws_bytes < plan->ws_bytes || !aligned16(lse_ws)) return PA_ERR_WORKSPACE;
+  if (!out || !aligned16(out)) return PA_ERR_INVALID_ARG;
+  thread_local SplitTable table;
+  for (size_t i = 0; i < sch.split.size(); ++i) table.blk[i] = sch.split[i];
+  for (size_t i = 0; i < bt.seq.size(); ++i) table.seq[i] = bt.seq[i];
+  const int D = plan->head_dim;
+  const int64_t warps = (int64_t)sch.split.size() * sch.rows_per_block;
+  combine_blocks_kernel<<<(unsigned)((warps + 7) / 8), 256, 0,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(
+      lse_ws, lse_ws + (int64_t)sch.n_slots * sch.rows_per_block * D, out, table,
+      (int)sch.split.size(), sch.rows_per_block, 0, plan->n_kv_heads, plan->group, 0,
+      plan->n_q_heads, D, (int)bt.seq.size());
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -101,23 +101,14 @@ namespace pa {
 // worker's share ends. Every worker then carries the same load and at most one cut per worker
 // boundary is made; no piece shorter than `m` tiles is cut off. Items are issued in the order of
 // their planned start, so the hardware's first-free-SM dispatch reproduces the plan.
-bool build_balanced(const pa_plan_t& p, Schedule* out) {
-  const CostModel cm(p.head_dim);
-  const int per = ctas_per_unit_for(p.head_dim);
-  const int slots = std::max(1, p.num_sms / per);
-  const int64_t q_units = ((int64_t)p.q_tiles + per - 1) / per;
-  const int Hkv = p.n_kv_heads;
-  const int64_t n_rb = q_units * Hkv;
-  if (n_rb > kMaxItems) return false;
-  std::vector<int64_t> len(n_rb);
+// len[rb] is the KV-tile count of row block rb; `order` lists the row blocks longest first.
+static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32_t>& order,
+                        int slots, int per, int head_dim, Schedule* out) {
+  const CostModel cm(head_dim);
+  const int64_t n_rb = (int64_t)len.size();
+  if (n_rb > kMaxItems || n_rb == 0) return false;
   double total = 0.0;
-  for (int64_t rb = 0; rb < n_rb; ++rb) {
-    int64_t qu;
-    int g;
-    rb_coords((int32_t)rb, q_units, Hkv, &qu, &g);
-    len[rb] = unit_kv_tiles(qu, per, p.q_tiles, p.chunk_rows, p.group, p.hist_len);
-    total += (double)len[rb];
-  }
+  for (int64_t x : len) total += (double)x;
   const double c_item = cm.unit_us / cm.tile_us;  // fixed cost of an item, in tiles
   struct Piece {
     int32_t rb, kt0, kt1, worker;
@@ -129,7 +120,7 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
     pieces.clear();
     int k = 0;
     double load = 0.0;
-    for (int64_t rb = 0; rb < n_rb; ++rb) {
+    for (int32_t rb : order) {
       int64_t o = 0, r = len[rb];
       while (r > 0) {
         const double room = share - load - c_item;
@@ -146,7 +137,7 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
           take = std::max<int64_t>((int64_t)room, m);
           if (r - take < m) take = r;
         }
-        pieces.push_back({(int32_t)rb, (int32_t)o, (int32_t)(o + take), k, load});
+        pieces.push_back({rb, (int32_t)o, (int32_t)(o + take), k, load});
         load += (double)take + c_item;
         o += take;
         r -= take;
@@ -161,6 +152,11 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
   // The smallest share (from the even split of the tiles plus one item cost per row block and
   // per cut) whose assignment fits the workers.
   double share = (total + c_item * (double)(n_rb + slots - 1)) / slots;
+  // no row block in more parts than the combine merges (a part may also start and end a worker
+  // part-way, hence one part of slack)
+  int64_t max_len = 0;
+  for (int64_t x : len) max_len = std::max(max_len, x);
+  share = std::max(share, (double)max_len / (PA_MAX_SPLITS - 2) + c_item + 1.0);
   const int64_t m = std::max<int64_t>(4, (int64_t)(share / 32.0));
   const double over = 1.0 + share / 128.0;
   for (int it = 0; it < 400 && assign(share, m, over) > slots; ++it) share *= 1.002;
@@ -182,19 +178,19 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
   }
   if ((int64_t)sch.split.size() > kMaxSplitBlocks || sch.max_parts > PA_MAX_SPLITS) return false;
   std::vector<int32_t> seen(n_rb, 0);
-  std::vector<std::pair<std::pair<double, int>, PaItem>> order;
+  std::vector<std::pair<std::pair<double, int>, PaItem>> items;
   for (const Piece& pc : pieces) {  // pieces of a row block appear in key order
     const int32_t slot = parts[pc.rb] > 1 ? first[pc.rb] + seen[pc.rb]++ : -1;
-    order.push_back({{pc.start, pc.worker}, PaItem{pc.rb, pc.kt0, pc.kt1, slot}});
+    items.push_back({{pc.start, pc.worker}, PaItem{pc.rb, pc.kt0, pc.kt1, slot}});
   }
-  std::stable_sort(order.begin(), order.end(),
+  std::stable_sort(items.begin(), items.end(),
                    [](const auto& x, const auto& y) { return x.first < y.first; });
-  for (const auto& o : order) sch.items.push_back(o.second);
+  for (const auto& o : items) sch.items.push_back(o.second);
   double comb = 0.0;
   if (!sch.split.empty()) {
     double bytes = 0.0;
     for (const PaSplitBlock& b : sch.split)
-      bytes += (double)(b.nparts + 1) * sch.rows_per_block * (p.head_dim + 1) * 4.0;
+      bytes += (double)(b.nparts + 1) * sch.rows_per_block * (head_dim + 1) * 4.0;
     comb = bytes * cm.combine_us_per_byte + cm.combine_fixed_us;
   }
   sch.makespan_us = simulate_items(sch.items, slots, cm) + comb;
@@ -202,7 +198,111 @@ bool build_balanced(const pa_plan_t& p, Schedule* out) {
   return true;
 }
 
+bool build_balanced(const pa_plan_t& p, Schedule* out) {
+  const int per = ctas_per_unit_for(p.head_dim);
+  const int slots = std::max(1, p.num_sms / per);
+  const int64_t q_units = ((int64_t)p.q_tiles + per - 1) / per;
+  const int Hkv = p.n_kv_heads;
+  const int64_t n_rb = q_units * Hkv;
+  if (n_rb > kMaxItems || n_rb <= 0) return false;
+  std::vector<int64_t> len(n_rb);
+  std::vector<int32_t> order(n_rb);
+  for (int64_t rb = 0; rb < n_rb; ++rb) {  // row-block numbering is already longest first
+    int64_t qu;
+    int g;
+    rb_coords((int32_t)rb, q_units, Hkv, &qu, &g);
+    len[rb] = unit_kv_tiles(qu, per, p.q_tiles, p.chunk_rows, p.group, p.hist_len);
+    order[rb] = (int32_t)rb;
+  }
+  return wrap_around(len, order, slots, per, p.head_dim, out);
+}
+
+int describe_batch(int batch, const int32_t* q_lens, const int64_t* hist_lens, int G, int Hkv,
+                   int per, Batch* out) {
+  if (batch <= 0 || !q_lens || !hist_lens || G <= 0 || Hkv <= 0) return PA_ERR_INVALID_ARG;
+  if (batch > kMaxSeqs) return PA_ERR_UNSUPPORTED;
+  Batch bt;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t r = q_lens[b], h = hist_lens[b];
+    if (r < 0 || h < 0) return PA_ERR_INVALID_ARG;
+    if (h + r + kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    const int64_t q_units = ceil_div64(q_tiles_for(r, G), per);
+    bt.seq.push_back({(int32_t)bt.total_rows, (int32_t)r, (int32_t)h, (int32_t)bt.row_blocks});
+    bt.total_rows += r;
+    bt.row_blocks += q_units * Hkv;
+    bt.max_hist = std::max(bt.max_hist, h);
+    if (bt.total_rows >= (int64_t(1) << 31) || bt.row_blocks > kMaxItems)
+      return PA_ERR_UNSUPPORTED;
+  }
+  if (bt.total_rows == 0) return PA_ERR_INVALID_ARG;
+  *out = std::move(bt);
+  return PA_OK;
+}
+
+bool build_batch(int num_sms, int head_dim, int G, int Hkv, const Batch& bt, Schedule* out) {
+  const int per = ctas_per_unit_for(head_dim);
+  const int slots = std::max(1, num_sms / per);
+  std::vector<int64_t> len;
+  for (const PaSeq& sq : bt.seq) {
+    const int64_t q_tiles = q_tiles_for(sq.rows, G);
+    const int64_t q_units = ceil_div64(q_tiles, per);
+    for (int64_t local = 0; local < q_units * Hkv; ++local) {
+      int64_t qu;
+      int g;
+      rb_coords((int32_t)local, q_units, Hkv, &qu, &g);
+      len.push_back(unit_kv_tiles(qu, per, q_tiles, sq.rows, G, sq.hist));
+    }
+  }
+  std::vector<int32_t> order(len.size());
+  for (size_t i = 0; i < order.size(); ++i) order[i] = (int32_t)i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int32_t x, int32_t y) { return len[x] > len[y]; });
+  return wrap_around(len, order, slots, per, head_dim, out);
+}
+
 }  // namespace pa
+
+extern "C" int pa_batch_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
+                             int page_size, int batch, const int32_t* q_lens,
+                             const int64_t* hist_lens, int dtype, float scale, pa_plan_t* plan) {
+  if (!plan) return PA_ERR_INVALID_ARG;
+  memset(plan, 0, sizeof *plan);
+  if (num_sms <= 0 || n_q_heads <= 0 || n_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || isinf(scale)) return PA_ERR_INVALID_ARG;
+  if (n_q_heads % n_kv_heads) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (!is_pow2(page_size) || page_size < 16 || page_size > 128) return PA_ERR_UNSUPPORTED;
+  const int G = n_q_heads / n_kv_heads;
+  const int per = ctas_per_unit_for(head_dim);
+  pa::Batch bt;
+  const int st = pa::describe_batch(batch, q_lens, hist_lens, G, n_kv_heads, per, &bt);
+  if (st != PA_OK) return st;
+  pa::Schedule sch;
+  if (!pa::build_batch(num_sms, head_dim, G, n_kv_heads, bt, &sch)) return PA_ERR_UNSUPPORTED;
+  int64_t q_tiles = 0;
+  for (const pa::PaSeq& sq : bt.seq) q_tiles += pa::q_tiles_for(sq.rows, G);
+  plan->num_sms = num_sms;
+  plan->n_q_heads = n_q_heads;
+  plan->n_kv_heads = n_kv_heads;
+  plan->head_dim = head_dim;
+  plan->page_size = page_size;
+  plan->group = G;
+  plan->chunk_rows = (int32_t)bt.total_rows;
+  plan->q_tiles = (int32_t)q_tiles;
+  plan->splits = sch.max_parts;
+  plan->paged = 1;
+  plan->dtype = dtype;
+  plan->policy = PA_POLICY_BALANCED;
+  plan->ctas_per_unit = per;
+  plan->batch = batch;
+  plan->hist_len = bt.max_hist;
+  plan->units = (int64_t)sch.items.size();
+  plan->scale = scale > 0.0f ? scale : (float)(1.0 / sqrt((double)head_dim));
+  plan->est_us = (float)sch.makespan_us;
+  plan->ws_bytes = (uint64_t)sch.n_slots * sch.rows_per_block * (head_dim + 1) * 4ull;
+  return PA_OK;
+}
 
 extern "C" int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
                               int page_size, int batch, int64_t max_seq_len, int dtype,
@@ -370,11 +470,7 @@ extern "C" int pa_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim,
   return PA_OK;
 }
 
-extern "C" int pa_schedule_items(const pa_plan_t* plan, int32_t* items, int cap) {
-  if (!plan || plan->policy != PA_POLICY_BALANCED) return 0;
-  pa::Schedule sch;
-  if (!pa::build_balanced(*plan, &sch) || (int64_t)sch.items.size() != plan->units)
-    return PA_ERR_INVALID_ARG;
+static int write_items(const pa::Schedule& sch, int32_t* items, int cap) {
   const int n = (int)sch.items.size();
   for (int i = 0; i < n && i < cap && items; ++i) {
     items[4 * i + 0] = sch.items[i].rb;
@@ -383,6 +479,29 @@ extern "C" int pa_schedule_items(const pa_plan_t* plan, int32_t* items, int cap)
     items[4 * i + 3] = sch.items[i].slot;
   }
   return n;
+}
+
+extern "C" int pa_batch_schedule_items(const pa_plan_t* plan, const int32_t* q_lens,
+                                       const int64_t* hist_lens, int32_t* items, int cap) {
+  if (!plan || plan->batch <= 0 || plan->policy != PA_POLICY_BALANCED) return PA_ERR_INVALID_ARG;
+  pa::Batch bt;
+  const int st = pa::describe_batch(plan->batch, q_lens, hist_lens, plan->group,
+                                    plan->n_kv_heads, plan->ctas_per_unit, &bt);
+  if (st != PA_OK) return st;
+  pa::Schedule sch;
+  if (!pa::build_batch(plan->num_sms, plan->head_dim, plan->group, plan->n_kv_heads, bt, &sch) ||
+      (int64_t)sch.items.size() != plan->units)
+    return PA_ERR_INVALID_ARG;
+  return write_items(sch, items, cap);
+}
+
+extern "C" int pa_schedule_items(const pa_plan_t* plan, int32_t* items, int cap) {
+  if (!plan || plan->policy != PA_POLICY_BALANCED) return 0;
+  if (plan->batch != 0) return PA_ERR_INVALID_ARG;  // pa_batch_schedule_items
+  pa::Schedule sch;
+  if (!pa::build_balanced(*plan, &sch) || (int64_t)sch.items.size() != plan->units)
+    return PA_ERR_INVALID_ARG;
+  return write_items(sch, items, cap);
 }
 
 extern "C" const char* pa_status_string(int status) {

@@ -46,8 +46,9 @@ template <bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_q, const PrefillArgs a,
+                        const __grid_constant__ CUtensorMap tm_q, const PrefillArgs a_in,
                         const __grid_constant__ ItemTable items) {
+  PrefillArgs a = a_in;  // rebased on one sequence in batched plans
   using C = PairCfg;
   constexpr int D = 256, NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
@@ -60,16 +61,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   int64_t tp, kt0, kt1;
   int g, s, slot = kSlotUniform;
-  const int64_t q_pairs = (a.q_tiles + 1) / 2;
   if (a.balanced) {
     const PaItem it = items.item[blockIdx.x >> 1];
-    rb_coords(it.rb, q_pairs, a.Hkv, &tp, &g);
+    const int32_t rb = a.batch > 0 ? batch_rebase<D>(a, items, it.rb) : it.rb;
+    rb_coords(rb, (a.q_tiles + 1) / 2, a.Hkv, &tp, &g);
     s = 0;
     kt0 = it.kt0;
     kt1 = it.kt1;
     slot = it.slot;
   } else {
-    unit_coords(blockIdx.x >> 1, q_pairs, a.Hkv, a.splits, &tp, &g, &s);
+    unit_coords(blockIdx.x >> 1, (a.q_tiles + 1) / 2, a.Hkv, a.splits, &tp, &g, &s);
     const int64_t qt_last = 2 * tp + 1 < a.q_tiles ? 2 * tp + 1 : a.q_tiles - 1;
     split_range(tile_kv_tiles(qt_last, a.R, a.G, a.hist_len), s, a.splits, &kt0, &kt1);
   }
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Q tile: four 16 KB panels of 128/G whole tokens; both CTAs' bytes complete on rank 0's
     // barrier, which rank 0 arms for both. Rows past the piece arrive as zeros.
     if (a.q_tma && w == 0 && lane == 0) {
-      const int32_t t0 = (int32_t)(qt * (kTileRows / a.G));
+      const int32_t t0 = a.q_row0 + (int32_t)(qt * (kTileRows / a.G));
       if (rank == 0) mbar_arrive_expect_tx(bar(C::B_QFULL), 2u * 4u * kPanel);
       for (int p = 0; p < 4; ++p) {
         if (rank == 0)

@@ -250,3 +250,36 @@ def _place(pool: np.ndarray, logical: np.ndarray, pages: np.ndarray, PS: int):
         pool[pages[:full]] = logical[:full * PS].reshape(full, PS, *logical.shape[1:])
     if n - full * PS:
         pool[pages[full], :n - full * PS] = logical[full * PS:]
+
+
+@dataclass
+class SeqBatch:
+    """A batch of chunks over one shared page pool (host side): sequence b has hist_lens[b]
+    keys of history and q_lens[b] query rows (whose K/V are in the pool too), on the pages
+    block_table[b, :ceil((hist + rows)/PS)]; its rows are q[q_row0[b] : q_row0[b] + q_lens[b]].
+    Pages of different sequences are disjoint; table padding is -1, unowned slots NaN."""
+    q: np.ndarray            # [sum q_lens, Hq, D]
+    k_pool: np.ndarray
+    v_pool: np.ndarray
+    block_table: np.ndarray  # int32 [B, max_pages]
+    q_lens: np.ndarray       # int32 [B]
+    hist_lens: np.ndarray    # int64 [B]
+    dtype: str
+    scale: float = 0.0
+
+    @property
+    def q_row0(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.q_lens)[:-1]]).astype(np.int64)
+
+
+def seq_batch(seed: int, hist_lens, q_lens, Hq: int, Hkv: int, D: int, PS: int, dtype: str,
+              pool_factor: float = 1.1, poison: bool = True) -> SeqBatch:
+    """Seeded N(0, 1) inputs for a batch of chunks: sequence b keeps hist_lens[b] + q_lens[b]
+    keys on its own shuffled pages of one pool."""
+    hist = np.asarray(hist_lens, dtype=np.int64)
+    rows = np.asarray(q_lens, dtype=np.int32)
+    keys = hist + rows
+    db = decode_batch(seed, keys, Hq, Hkv, D, PS, dtype, pool_factor, poison)
+    rng = np.random.default_rng(seed + 7)
+    q = to_bits(rng.standard_normal((int(rows.sum()), Hq, D), dtype=np.float32), dtype)
+    return SeqBatch(q, db.k_pool, db.v_pool, db.block_table, rows, hist, dtype)
