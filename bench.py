@@ -191,13 +191,15 @@ def time_steps(dw, steps, warmup, flush, stream, record_kernels=False):
     import torch
     from paged_kv_long_b200 import binding
     for _ in range(warmup):
-        flush.zero_()
+        with torch.cuda.stream(stream):
+            flush.zero_()
         dw.run(stream)
     torch.cuda.synchronize()
     step_ms, kern_ms = [], []
     evs = []
     for _ in range(steps):
-        flush.zero_()
+        with torch.cuda.stream(stream):  # on the timed stream: done before the step's events
+            flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         kev = []
@@ -338,6 +340,39 @@ def decode_measure(wl, dev, stream, peaks, reps=20, seed=6000):
                          "frac": nbytes / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
 
 
+def routes_measure(inp, dev, stream, flush, reps=8):
+    """The cold prompt's two bulk-prefill routes, each a whole step (every chunk): paged (append
+    the chunk's K/V to pages, prefill through the table) and contiguous staging + page publish
+    (prefill on the staging buffer, publish the chunk's rows). L2 flushed before each step; the
+    two routes' steps alternate and each route reports its median."""
+    import torch
+    from paged_kv_long_b200.runner import PrefillRoutes
+    rt = PrefillRoutes(inp, dev)
+    routes = (("paged", rt.run_paged), ("staged", rt.run_staged))
+    evs = {r: [] for r, _ in routes}
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for _, fn in routes:
+                fn(stream)
+        for _ in range(reps):  # interleaved, so that drift hits both routes alike
+            for route, fn in routes:
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn(stream)
+                e1.record(stream)
+                evs[route].append((e0, e1))
+        torch.cuda.synchronize()
+    res = {r: statistics.median(a.elapsed_time(b) for a, b in e) for r, e in evs.items()}
+    same = all(torch.equal(a, b) for a, b in zip(rt.outs["paged"], rt.outs["staged"]))
+    del rt
+    return {"workload": "cold prompt of the bench workload, chunk by chunk",
+            "paged_route_ms": res["paged"], "staged_route_ms": res["staged"],
+            "staged_over_paged_time": res["staged"] / res["paged"],
+            "outputs_identical": bool(same)}
+
+
 def e2e_steps(inp, dw, steps, stream):
     """End to end through the public API: pinned host inputs -> device, prefill + combine for
     every piece, outputs -> pinned host, every step. Returns (per-step ms, h2d, d2h bytes)."""
@@ -431,7 +466,7 @@ def gpu_arm(args):
     t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
 
     # ---- contiguous control at the same split counts (the ratio's denominator)
-    t_contig = last_paged = last_contig = None
+    t_contig = t_paged_pairs = last_paged = last_contig = None
     if paged and not args.no_contiguous:
         from paged_kv_long_b200 import binding
         # the same schedule per piece as the paged run (the planner does not look at the layout)
@@ -439,17 +474,31 @@ def gpu_arm(args):
         for p, pc in zip(dw.plans, dwc.plans):
             assert (p.policy, p.splits, p.units, p.ws_bytes) == (pc.policy, pc.splits, pc.units,
                                                                 pc.ws_bytes)
-        c_ms, c_kern = time_steps(dwc, max(3, args.steps // 2), args.warmup, flush, stream,
-                                  record_kernels=True)
-        t_contig = sum(c_ms) / len(c_ms)
-        last_paged = statistics.median(k[-1] for k in kern_ms)
-        last_contig = statistics.median(k[-1] for k in c_kern)
+        # paged and contiguous steps alternate, so that clock or neighbour drift hits both
+        time_steps(dwc, 0, args.warmup, flush, stream)
+        pp, cc, pk, ck = [], [], [], []
+        for _ in range(max(6, args.steps // 2)):
+            a_ms, a_k = time_steps(dw, 1, 0, flush, stream, record_kernels=True)
+            b_ms, b_k = time_steps(dwc, 1, 0, flush, stream, record_kernels=True)
+            pp += a_ms
+            cc += b_ms
+            pk.append(a_k[0][-1])
+            ck.append(b_k[0][-1])
+        t_paged_pairs = statistics.median(pp)
+        t_contig = statistics.median(cc)
+        last_paged = statistics.median(pk)
+        last_contig = statistics.median(ck)
         del dwc
 
     # ---- KV append, the step before prefill (its own HBM roofline)
     kv = None
     if paged and not args.no_kv_append:
         kv = kv_append_measure(inp, dev, stream, peaks)
+
+    # ---- contiguous staging + page publish against the paged route (cold prompts only)
+    routes = None
+    if paged and not args.no_routes and wl.first_pos == 0:
+        routes = routes_measure(inp, dev, stream, flush)
 
     # ---- batched paged decode on a cache of the same shape (its own HBM roofline)
     dec = None
@@ -491,9 +540,10 @@ def gpu_arm(args):
                    "l2": f"flushed between steps ({args.l2_flush_mb} MiB write outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "tflops": tflops,
-        "paged_contiguous_ratio": (t_contig / t_step) if t_contig else None,
+        "paged_contiguous_ratio": (t_contig / t_paged_pairs) if t_contig else None,
         "paged_contiguous_ratio_last_chunk": (last_contig / last_paged) if t_contig else None,
         "contiguous_ms_per_step": t_contig,
+        "ratio_method": "median of alternating paged / contiguous steps (L2 flushed before each)",
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": None,
                      "peak_source": f"{peaks['source']} bf16 dense (burst)",
@@ -503,6 +553,7 @@ def gpu_arm(args):
         "e2e": e2e,
         "kv_append": kv,
         "decode": dec,
+        "staging_route": routes,
         "cpu_baseline": cpu,
         "gpu_launches": launches,
         "clocks": clocks,
@@ -528,6 +579,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-kv-append", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-routes", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)

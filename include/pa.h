@@ -309,6 +309,18 @@ int pa_kv_append(int n_kv_heads, int head_dim, int page_size, int dtype, const v
                  int64_t num_pages, int64_t hist_len, int chunk_rows, pa_stream_t stream);
 
 /*
+ * pa_kv_publish — the page publish of the contiguous-staging route (BaseRT issue #51,
+ * "Expected vs actual": bulk prefill on a contiguous staging buffer, completed K/V then
+ * published to pages). Copies staged rows [first_pos, first_pos + rows) of
+ * k_staged / v_staged (device [T][Hkv][D], the prompt's positions from 0) to their pages:
+ * position p goes to page page_table[p/PS], slot p%PS. Same kernel, checks and errors as
+ * pa_kv_append (whose k_new is the staged buffer advanced by first_pos rows).
+ */
+int pa_kv_publish(int n_kv_heads, int head_dim, int page_size, int dtype, const void* k_staged,
+                  const void* v_staged, void* k_pool, void* v_pool, const int32_t* page_table,
+                  int64_t num_pages, int64_t first_pos, int rows, pa_stream_t stream);
+
+/*
  * pa_device_error — synchronise the current device, then read (and with reset != 0,
  * clear) the library's device-side error word. *flags receives its bits
  * (1: page index out of range, 2: a wait timed out). Returns PA_OK when no bit is set,

@@ -24,7 +24,7 @@ EXPORTED = ("pa_plan", "pa_prefill", "pa_combine", "pa_prefill_noalloc", "pa_dev
             "pa_selftest_timeout", "pa_status_string", "pa_cores_policy_splits",
             "pa_legacy_policy_splits", "pa_schedule_items", "pa_kv_append", "pa_pieces",
             "pa_decode_plan", "pa_decode", "pa_batch_plan", "pa_batch_prefill",
-            "pa_batch_combine", "pa_batch_schedule_items")
+            "pa_batch_combine", "pa_batch_schedule_items", "pa_kv_publish")
 
 
 class PaError(RuntimeError):
@@ -109,6 +109,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.pa_batch_schedule_items.argtypes = [ctypes.POINTER(Plan), vp, vp,
                                             ctypes.POINTER(ctypes.c_int32), i32]
     lib.pa_batch_schedule_items.restype = i32
+    lib.pa_kv_publish.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i64, i32, vp]
+    lib.pa_kv_publish.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -190,6 +192,36 @@ def kv_append(k_new, v_new, k_pool, v_pool, page_table, hist_len: int, stream=No
                                      page_table.data_ptr(), k_pool.shape[0], hist_len, R,
                                      _stream_ptr(stream))
     _check(st, "pa_kv_append")
+
+
+def kv_publish(k_staged, v_staged, k_pool, v_pool, page_table, first_pos: int, rows: int,
+               stream=None):
+    """pa_kv_publish: copy staged rows [first_pos, first_pos + rows) of the contiguous staging
+    buffers [T, Hkv, D] to their pages (see include/pa.h)."""
+    import torch
+    if k_staged.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("k_staged must be float16 or bfloat16")
+    dt = k_staged.dtype
+    _require_cuda(k_staged, "k_staged", dt)
+    if k_staged.dim() != 3:
+        raise ValueError("k_staged must be [T, Hkv, D]")
+    T, Hkv, D = k_staged.shape
+    if first_pos < 0 or rows < 0 or first_pos + rows > T:
+        raise ValueError("rows [first_pos, first_pos + rows) must lie in the staging buffer")
+    _require_cuda(v_staged, "v_staged", dt, (T, Hkv, D))
+    _require_cuda(k_pool, "k_pool", dt)
+    if k_pool.dim() != 4 or tuple(k_pool.shape[2:]) != (Hkv, D):
+        raise ValueError("k_pool must be [num_pages, page_size, Hkv, D]")
+    _require_cuda(v_pool, "v_pool", dt, tuple(k_pool.shape))
+    _require_cuda(page_table, "page_table", torch.int32)
+    PS = k_pool.shape[1]
+    if page_table.numel() < math.ceil((first_pos + rows) / PS):
+        raise ValueError("page_table is shorter than ceil((first_pos+rows)/page_size)")
+    st = load_library().pa_kv_publish(Hkv, D, PS, _dtype_code(dt), k_staged.data_ptr(),
+                                      v_staged.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                      page_table.data_ptr(), k_pool.shape[0], first_pos, rows,
+                                      _stream_ptr(stream))
+    _check(st, "pa_kv_publish")
 
 
 def _stream_ptr(stream):

@@ -1292,16 +1292,19 @@ namespace pa {
 // The batch and its schedule, rebuilt from the caller's lengths and checked against the plan.
 static int rebuild_batch(const pa_plan_t* plan, const int32_t* q_lens, const int64_t* hist_lens,
                          Batch* bt, Schedule* sch) {
-  if (!plan || plan->batch <= 0 || plan->policy != PA_POLICY_BALANCED) return PA_ERR_INVALID_ARG;
+  if (!plan || plan->batch <= 0 || plan->policy != PA_POLICY_BALANCED || !q_lens || !hist_lens)
+    return PA_ERR_INVALID_ARG;
+  if (plan->batch > kMaxSeqs) return PA_ERR_UNSUPPORTED;
   const int D = plan->head_dim;
   if (D != 64 && D != 128 && D != 256) return PA_ERR_UNSUPPORTED;
   if (plan->n_kv_heads <= 0 || plan->n_q_heads != plan->n_kv_heads * plan->group ||
-      plan->ctas_per_unit != (D == 256 ? 2 : 1))
+      plan->ctas_per_unit != batch_ctas_per_unit(D, plan->group, plan->batch, q_lens))
     return PA_ERR_INVALID_ARG;
   const int st = describe_batch(plan->batch, q_lens, hist_lens, plan->group, plan->n_kv_heads,
                                 plan->ctas_per_unit, bt);
   if (st != PA_OK) return st;
-  if (!build_batch(plan->num_sms, D, plan->group, plan->n_kv_heads, *bt, sch) ||
+  if (!build_batch(plan->num_sms, D, plan->ctas_per_unit, plan->group, plan->n_kv_heads, *bt,
+                   sch) ||
       (int64_t)sch->items.size() != plan->units || bt->total_rows != plan->chunk_rows ||
       (uint64_t)sch->n_slots * sch->rows_per_block * (D + 1) * 4ull != plan->ws_bytes)
     return PA_ERR_INVALID_ARG;
@@ -1379,8 +1382,12 @@ extern "C" int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens,
     case 64: e = launch_d<64>(true, bf16, grid, cs, tk, tv, a, table); break;
     case 128: e = launch_d<128>(true, bf16, grid, cs, tk, tv, a, table); break;
     default:
-      e = bf16 ? launch_pair<true, true>(grid, cs, tk, tv, tq, a, table)
-               : launch_pair<true, false>(grid, cs, tk, tv, tq, a, table);
+      if (per == 2)
+        e = bf16 ? launch_pair<true, true>(grid, cs, tk, tv, tq, a, table)
+                 : launch_pair<true, false>(grid, cs, tk, tv, tq, a, table);
+      else
+        e = bf16 ? launch_prefill<256, true, true>(grid, cs, tk, tv, a, table)
+                 : launch_prefill<256, true, false>(grid, cs, tk, tv, a, table);
       break;
   }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -1474,6 +1481,18 @@ extern "C" int pa_kv_append(int n_kv_heads, int head_dim, int page_size, int dty
       static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), page_table, num_pages, hist_len,
       chunk_rows, page_size, row_vecs);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_kv_publish(int n_kv_heads, int head_dim, int page_size, int dtype,
+                             const void* k_staged, const void* v_staged, void* k_pool,
+                             void* v_pool, const int32_t* page_table, int64_t num_pages,
+                             int64_t first_pos, int rows, pa_stream_t stream) {
+  if (!k_staged || !v_staged || first_pos < 0) return PA_ERR_INVALID_ARG;
+  const int64_t off = first_pos * n_kv_heads * head_dim * 2;  // bytes of the rows before
+  return pa_kv_append(n_kv_heads, head_dim, page_size, dtype,
+                      static_cast<const uint8_t*>(k_staged) + off,
+                      static_cast<const uint8_t*>(v_staged) + off, k_pool, v_pool, page_table,
+                      num_pages, first_pos, rows, stream);
 }
 
 extern "C" int pa_device_error(int* flags, int reset) {

@@ -239,8 +239,14 @@ int describe_batch(int batch, const int32_t* q_lens, const int64_t* hist_lens, i
   return PA_OK;
 }
 
-bool build_batch(int num_sms, int head_dim, int G, int Hkv, const Batch& bt, Schedule* out) {
-  const int per = ctas_per_unit_for(head_dim);
+int batch_ctas_per_unit(int head_dim, int G, int batch, const int32_t* q_lens) {
+  int64_t max_qt = 0;
+  for (int b = 0; b < batch; ++b) max_qt = std::max(max_qt, q_tiles_for(q_lens[b], G));
+  return head_dim == 256 && max_qt > 1 ? 2 : 1;
+}
+
+bool build_batch(int num_sms, int head_dim, int per, int G, int Hkv, const Batch& bt,
+                 Schedule* out) {
   const int slots = std::max(1, num_sms / per);
   std::vector<int64_t> len;
   for (const PaSeq& sq : bt.seq) {
@@ -274,12 +280,17 @@ extern "C" int pa_batch_plan(int num_sms, int n_q_heads, int n_kv_heads, int hea
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
   if (!is_pow2(page_size) || page_size < 16 || page_size > 128) return PA_ERR_UNSUPPORTED;
   const int G = n_q_heads / n_kv_heads;
-  const int per = ctas_per_unit_for(head_dim);
+  if (batch <= 0 || !q_lens || !hist_lens) return PA_ERR_INVALID_ARG;
+  for (int b = 0; b < batch; ++b)
+    if (q_lens[b] < 0) return PA_ERR_INVALID_ARG;
+  // CTA pairs only when some sequence has two Q tiles to pair; else one CTA per row block
+  const int per = pa::batch_ctas_per_unit(head_dim, G, batch, q_lens);
   pa::Batch bt;
   const int st = pa::describe_batch(batch, q_lens, hist_lens, G, n_kv_heads, per, &bt);
   if (st != PA_OK) return st;
   pa::Schedule sch;
-  if (!pa::build_batch(num_sms, head_dim, G, n_kv_heads, bt, &sch)) return PA_ERR_UNSUPPORTED;
+  if (!pa::build_batch(num_sms, head_dim, per, G, n_kv_heads, bt, &sch))
+    return PA_ERR_UNSUPPORTED;
   int64_t q_tiles = 0;
   for (const pa::PaSeq& sq : bt.seq) q_tiles += pa::q_tiles_for(sq.rows, G);
   plan->num_sms = num_sms;
@@ -489,7 +500,8 @@ extern "C" int pa_batch_schedule_items(const pa_plan_t* plan, const int32_t* q_l
                                     plan->n_kv_heads, plan->ctas_per_unit, &bt);
   if (st != PA_OK) return st;
   pa::Schedule sch;
-  if (!pa::build_batch(plan->num_sms, plan->head_dim, plan->group, plan->n_kv_heads, bt, &sch) ||
+  if (!pa::build_batch(plan->num_sms, plan->head_dim, plan->ctas_per_unit, plan->group,
+                       plan->n_kv_heads, bt, &sch) ||
       (int64_t)sch.items.size() != plan->units)
     return PA_ERR_INVALID_ARG;
   return write_items(sch, items, cap);

@@ -32,7 +32,11 @@ struct Batch {
 // Validates the lengths and lays the sequences out (rows packed in order). Returns a pa_status.
 int describe_batch(int batch, const int32_t* q_lens, const int64_t* hist_lens, int G, int Hkv,
                    int per, Batch* out);
+// CTAs per row block of a batch: 2 (CTA pairs, head dim 256) only when some sequence has two
+// or more Q tiles; a batch of one-tile sequences (decode) would leave half of every pair idle.
+int batch_ctas_per_unit(int head_dim, int G, int batch, const int32_t* q_lens);
 // The balanced schedule of a batch (row blocks of all sequences, longest first).
-bool build_batch(int num_sms, int head_dim, int G, int Hkv, const Batch& bt, Schedule* out);
+bool build_batch(int num_sms, int head_dim, int per, int G, int Hkv, const Batch& bt,
+                 Schedule* out);
 
 }  // namespace pa

@@ -67,3 +67,65 @@ class DeviceWorkload:
 
     def outputs_host(self) -> list[np.ndarray]:
         return [o.cpu().numpy() for o in self.outs]
+
+
+class PrefillRoutes:
+    """The two bulk-prefill routes of a cold prompt (history 0, chunks in order), with the same
+    plans' schedules and the same outputs:
+
+    * paged (the hot path): each chunk's K/V, as the projection leaves them in a contiguous
+      [R, Hkv, D] buffer, are appended to their pages (pa_kv_append), then prefill reads every
+      key through the page table;
+    * staged: the projection writes each chunk's K/V straight into a contiguous staging buffer
+      [T, Hkv, D] at the chunk's positions, prefill reads the staged keys contiguously, and the
+      chunk's rows are then published to their pages (pa_kv_publish).
+
+    Both leave the same page pools behind. ``k_new``/``v_new`` stand for the projection's output
+    (the staged route's staging buffer holds the same rows)."""
+
+    def __init__(self, inp: Inputs, device="cuda", policy: str = "makespan",
+                 num_sms: int | None = None):
+        import torch
+        wl = inp.wl
+        assert wl.first_pos == 0, "the routes start from an empty cache"
+        self.wl, self.device = wl, torch.device(device)
+        self.q = _dev_tensor(inp.q, wl.dtype, self.device)
+        self.kv_new = (_dev_tensor(inp.k_logical, wl.dtype, self.device),
+                       _dev_tensor(inp.v_logical, wl.dtype, self.device))
+        self.staged = (self.kv_new[0].clone(), self.kv_new[1].clone())
+        shape = inp.k_pool.shape
+        dt = self.q.dtype
+        self.pools = {r: (torch.zeros(shape, dtype=dt, device=self.device),
+                          torch.zeros(shape, dtype=dt, device=self.device))
+                      for r in ("paged", "staged")}
+        self.table = torch.from_numpy(inp.page_table).to(self.device)
+        self.plans = {}
+        for route, paged in (("paged", True), ("staged", False)):
+            self.plans[route] = [binding.plan(wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                                              wl.page_size, r, h, wl.dtype, wl.scale, 0, policy,
+                                              paged, num_sms) for h, r in wl.pieces]
+        self.outs = {r: [torch.empty((n, wl.n_q_heads, wl.head_dim), dtype=torch.float32,
+                                     device=self.device) for _, n in wl.pieces]
+                     for r in ("paged", "staged")}
+        ws = max(p.ws_bytes for ps in self.plans.values() for p in ps) // 4
+        self.ws = torch.empty(max(ws, 4), dtype=torch.float32, device=self.device)
+
+    def run_paged(self, stream=None):
+        kp, vp = self.pools["paged"]
+        for i, (h, r) in enumerate(self.wl.pieces):
+            binding.kv_append(self.kv_new[0][h:h + r], self.kv_new[1][h:h + r], kp, vp,
+                              self.table, h, stream)
+            p = self.plans["paged"][i]
+            binding.prefill(p, self.q[h:h + r], kp, vp, self.table, self.outs["paged"][i],
+                            self.ws, stream)
+            binding.combine(p, self.ws, self.outs["paged"][i], stream)
+
+    def run_staged(self, stream=None):
+        kp, vp = self.pools["staged"]
+        ks, vs = self.staged
+        for i, (h, r) in enumerate(self.wl.pieces):
+            p = self.plans["staged"][i]
+            binding.prefill(p, self.q[h:h + r], ks[:h + r], vs[:h + r], None,
+                            self.outs["staged"][i], self.ws, stream)
+            binding.combine(p, self.ws, self.outs["staged"][i], stream)
+            binding.kv_publish(ks, vs, kp, vp, self.table, h, r, stream)

@@ -138,7 +138,8 @@ def test_batch_schedule_covers_every_tile_once(seed):
         q_lens[:] = 1  # decode-like
     hist = rng.integers(0, 40000, size=B)
     num_sms = int(rng.choice([148, 132, 16, 7]))
-    per = 2 if D == 256 else 1
+    # CTA pairs at head dim 256 unless every sequence fits one Q tile
+    per = 2 if D == 256 and max(math.ceil(r * G / TILE) for r in q_lens) > 1 else 1
     tiles = row_block_tiles(q_lens, hist, Hkv, G, per)
     try:
         bp = bd.batch_plan(G * Hkv, Hkv, D, 16, q_lens, hist, "bf16", num_sms=num_sms)
@@ -146,12 +147,23 @@ def test_batch_schedule_covers_every_tile_once(seed):
         # the item table holds 512: row blocks plus at most one cut per worker must fit
         assert bd.STATUS[e.status] == "PA_ERR_UNSUPPORTED" and len(tiles) > 512 - num_sms // per
         return
+    assert bp.plan.ctas_per_unit == per
     items = bd.batch_schedule_items(bp)
     assert len(items) == bp.plan.units
     check_items(items, tiles, per * TILE)
     assert bp.plan.chunk_rows == q_lens.sum() and bp.plan.batch == B
     n_slots = sum(1 for it in items if it[3] >= 0)
     assert bp.plan.ws_bytes == n_slots * per * TILE * (D + 1) * 4
+
+
+def test_batch_pairs_only_when_a_sequence_has_two_q_tiles():
+    bd = _bd()
+    one = bd.batch_plan(16, 2, 256, 16, [1, 16, 3], [900, 20, 5000], "f16", num_sms=148)
+    assert one.plan.ctas_per_unit == 1            # 16 rows x 8 heads = one 128-row tile
+    two = bd.batch_plan(16, 2, 256, 16, [1, 17, 3], [900, 20, 5000], "f16", num_sms=148)
+    assert two.plan.ctas_per_unit == 2
+    small_d = bd.batch_plan(16, 2, 128, 16, [500, 17], [900, 20], "f16", num_sms=148)
+    assert small_d.plan.ctas_per_unit == 1
 
 
 def test_batch_schedule_balances_the_sms():
