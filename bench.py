@@ -416,6 +416,27 @@ def e2e_steps(inp, dw, steps, stream):
     return ms, h2d, d2h
 
 
+def section_arm(args):
+    """One side measurement alone (for profiling it): prints its JSON object on one line."""
+    import torch
+    from paged_kv_long_b200.inputs import WORKLOADS, generate
+    wl = WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(dev)
+    peaks = load_peaks()
+    if args.section == "decode":
+        res = decode_measure(wl, dev, stream, peaks, reps=args.steps)
+    else:
+        inp = generate(wl, poison=False)
+        if args.section == "kv_append":
+            res = kv_append_measure(inp, dev, stream, peaks, reps=args.steps)
+        else:
+            flush = torch.empty((L2_FLUSH_BYTES) // 4, dtype=torch.float32, device=dev)
+            res = routes_measure(inp, dev, stream, flush, reps=args.steps)
+    print(json.dumps({"section": args.section, **res}), flush=True)
+    return 0
+
+
 def gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -582,6 +603,8 @@ def main(argv=None):
     ap.add_argument("--no-kv-append", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-routes", action="store_true")
+    ap.add_argument("--section", default="all", choices=["all", "decode", "kv_append", "routes"],
+                    help="run one side measurement alone (1 GPU; --steps = its repetitions)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
@@ -589,6 +612,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args)
+    if args.section != "all":
+        return section_arm(args)
     return gpu_arm(args)
 
 
