@@ -107,6 +107,24 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest of every rank's x (a time: the job ends when its slowest replica does); x
+    itself without a process group. Every rank must call it, in the same order."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: float, t_ms: float) -> float:
+    """Whole-job rate of `world` replicas that each process units_per_rank units in at most
+    t_ms (the max over ranks)."""
+    return world * units_per_rank / (t_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- CPU oracle legs
 class OracleSampler:
     """The fp64 CPU oracle timed on a stride sample of (row, head) pairs spread over the whole
@@ -472,13 +490,9 @@ def gpu_arm(args):
         barrier()
         wall = time.perf_counter() - wall0
     clocks = clk.summary()
-    t_step = sum(step_ms) / len(step_ms)
-    if world > 1:
-        tt = torch.tensor([t_step], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step = float(tt.item())
+    t_step = max_over_ranks(sum(step_ms) / len(step_ms), dev)
     tokens = wl.query_rows
-    value = world * tokens / (t_step / 1e3)
+    value = job_throughput(world, tokens, t_step)
     flops = wl.flops()
     tflops = flops / (t_step / 1e3) / 1e12
 
@@ -532,8 +546,8 @@ def gpu_arm(args):
     e2e = None
     if not args.no_e2e and paged:
         e_ms, h2d, d2h = e2e_steps(inp, dw, max(2, min(args.steps, 5)), stream)
-        t_e = sum(e_ms) / len(e_ms)
-        e2e = {"value": world * tokens / (t_e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        t_e = max_over_ranks(sum(e_ms) / len(e_ms), dev)
+        e2e = {"value": job_throughput(world, tokens, t_e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": t_e}
 
     launches = args.steps * sum(1 + (1 if p.splits > 1 else 0) for p in dw.plans)
