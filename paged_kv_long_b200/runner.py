@@ -68,6 +68,45 @@ class DeviceWorkload:
     def outputs_host(self) -> list[np.ndarray]:
         return [o.cpu().numpy() for o in self.outs]
 
+    def run_streamed(self, host_q, host_k, host_v, host_table, host_outs, copy_in, compute,
+                     copy_out):
+        """One step from pinned host memory to pinned host memory with the copies overlapped:
+        the K/V pools and the page table go first (every chunk reads pages all over the pool);
+        then chunk i's query rows are copied on `copy_in` while earlier chunks compute on
+        `compute`, and chunk i's output goes back on `copy_out` while later chunks compute.
+        host_q [rows, Hq, D], host_k / host_v like the device pools, host_table int32,
+        host_outs: one pinned fp32 tensor per chunk. Enqueues only; returns the event that
+        completes with the last output copy."""
+        import torch
+        wl = self.wl
+        compute.wait_stream(copy_out)  # the previous step's outputs have left
+        with torch.cuda.stream(copy_in):
+            self.k.copy_(host_k, non_blocking=True)
+            self.v.copy_(host_v, non_blocking=True)
+            if self.table is not None:
+                self.table.copy_(host_table, non_blocking=True)
+        done = None
+        for i, (h, r) in enumerate(wl.pieces):
+            off = h - wl.first_pos
+            with torch.cuda.stream(copy_in):
+                self.q[off:off + r].copy_(host_q[off:off + r], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(copy_in)
+            compute.wait_event(ready)
+            self.run_piece(i, compute)
+            out_ready = torch.cuda.Event()
+            out_ready.record(compute)
+            copy_out.wait_event(out_ready)
+            with torch.cuda.stream(copy_out):
+                host_outs[i].copy_(self.outs[i], non_blocking=True)
+                done = torch.cuda.Event(enable_timing=True)
+                done.record(copy_out)
+        # the next step's copies into q / the pools must not overtake this step's reads
+        compute_done = torch.cuda.Event()
+        compute_done.record(compute)
+        copy_in.wait_event(compute_done)
+        return done
+
 
 class PrefillRoutes:
     """The two bulk-prefill routes of a cold prompt (history 0, chunks in order), with the same

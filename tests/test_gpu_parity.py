@@ -239,3 +239,37 @@ def test_c5_full_size_sampled_paged_equals_contiguous():
     _, outc = U.run_gpu(inp, paged=False)
     for a, b in zip(outs, outc):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+def test_gpu_streamed_step_equals_the_plain_step():
+    """DeviceWorkload.run_streamed (copies overlapped with compute on three streams, pinned host
+    buffers in and out) gives the plain run's outputs bit for bit, two steps back to back."""
+    import numpy as np
+    import torch
+    wl = U.custom_workload("streamed", 16, 2, 256, 16, "f16", [(0, 700), (700, 900), (1600, 513)],
+                           seed=8800)
+    inp = U.gen(wl, poison=True)
+    dw, want = U.run_gpu(inp)
+
+    def pinned(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if dt is not None:
+            t = t.view(torch.int16).view(dt)
+        return t.pin_memory()
+
+    hq = pinned(inp.q.view(np.int16), torch.float16)
+    hk = pinned(inp.k_pool.view(np.int16), torch.float16)
+    hv = pinned(inp.v_pool.view(np.int16), torch.float16)
+    ht = pinned(inp.page_table)
+    for o in dw.outs:
+        o.fill_(float("nan"))
+    houts = [torch.full(tuple(o.shape), float("nan")).pin_memory() for o in dw.outs]
+    s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    dw.run_streamed(hq, hk, hv, ht, houts, s_in, s_c, s_out)
+    done = dw.run_streamed(hq, hk, hv, ht, houts, s_in, s_c, s_out)
+    done.synchronize()
+    torch.cuda.synchronize()
+    for i, (h, w) in enumerate(zip(houts, want)):
+        assert np.array_equal(h.numpy(), w), f"piece {i}"
