@@ -31,6 +31,26 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 L2_FLUSH_BYTES = 512 << 20
 
 
+# DRAM traffic of the roofline kernel, per launch, from one ncu capture of the c5 bench step
+# (profiles/prefill_pair_kernel_c5_traffic.md: dram__bytes_read.sum + dram__bytes_write.sum
+# over the timed step's 16 launches / 16). It stands for the kernel whose sources hash to
+# `sources`; after any change to them the bench reports null until it is captured again.
+TRAFFIC_CAPTURE = {"workload": "c5", "sources": "815437c5a84d906b", "bytes_per_launch": 107.38e6}
+
+
+def kernel_sources_hash() -> str:
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "paged_kv_long_b200", "csrc", "*")) +
+                   [os.path.join(ROOT, "include", "pa.h")])
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -498,6 +518,13 @@ def gpu_arm(args):
     peak = peaks["bf16_tflops"]
     t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
 
+    traffic, traffic_note = None, "no capture of this kernel build"
+    if (paged and args.workload == TRAFFIC_CAPTURE["workload"] and args.policy == "makespan"
+            and args.splits is None and kernel_sources_hash() == TRAFFIC_CAPTURE["sources"]):
+        traffic = TRAFFIC_CAPTURE["bytes_per_launch"]
+        traffic_note = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, mean over the 16 "
+                        "launches of one step (cold L2 per launch under ncu), bytes per launch")
+
     # ---- contiguous control at the same split counts (the ratio's denominator)
     t_contig = t_paged_pairs = last_paged = last_contig = None
     if paged and not args.no_contiguous:
@@ -581,7 +608,8 @@ def gpu_arm(args):
         "contiguous_ms_per_step": t_contig,
         "ratio_method": "median of alternating paged / contiguous steps (L2 flushed before each)",
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak,
-                     "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": traffic,
+                     "traffic_source": traffic_note,
                      "peak_source": f"{peaks['source']} bf16 dense (burst)",
                      "step_frac_of_roofline": t_roof / (t_step / 1e3),
                      "kernel": "prefill_pair_kernel (pa_prefill, head dim 256)" if wl.head_dim == 256 else "prefill_kernel (pa_prefill)",
