@@ -150,10 +150,10 @@ class OracleSampler:
     """The fp64 CPU oracle timed on a stride sample of (row, head) pairs spread over the whole
     workload (one random head per sampled row), scaled to query tokens/s."""
 
-    def __init__(self, wl, inp):
+    def __init__(self, wl, inp, threads: int = 0):
         from oracle import oracle
         self.oracle, self.wl, self.inp = oracle, wl, inp
-        self.threads = oracle.max_threads()
+        self.threads = threads if threads > 0 else oracle.max_threads()
 
     def run(self, n: int, seed: int = 17):
         import numpy as np
@@ -172,7 +172,7 @@ class OracleSampler:
             pb = oracle.Problem(q=inp.piece_q(i), k=inp.k_pool, v=inp.v_pool, hist_len=h,
                                 dtype=wl.dtype, page_table=inp.page_table, scale=wl.scale)
             t0 = time.perf_counter()
-            oracle.attend(pb, sel, heads)
+            oracle.attend(pb, sel, heads, threads=self.threads)
             t_sum += time.perf_counter() - t0
             pairs += len(sel)
         # one (row, head) pair is 1/Hq of a query token's attention
@@ -198,7 +198,7 @@ def reference_arm(args):
     inp = generate(wl, poison=False)
     steps, warmup = args.steps, args.warmup
     per_step = max(1.0, min(10.0, 80.0 / max(steps + warmup, 1)))
-    sampler = OracleSampler(wl, inp)
+    sampler = OracleSampler(wl, inp, args.cpu_threads)
     n = sampler.calibrate(per_step)
     for k in range(warmup):
         sampler.run(max(8, n // 4), seed=50 + k)
@@ -580,7 +580,7 @@ def gpu_arm(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sampler = OracleSampler(wl, inp)
+        sampler = OracleSampler(wl, inp, args.cpu_threads)
         r, pairs, t = sampler.run(sampler.calibrate(args.cpu_seconds))
         cpu = {"value": r, "unit": UNIT, "cores": sampler.threads, "kind": "oracle",
                "sample": f"{pairs} (row, head) pairs stride-sampled over all {wl.query_rows} query "
@@ -648,6 +648,8 @@ def main(argv=None):
                     help="run one side measurement alone (1 GPU; --steps = its repetitions)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="host threads of the oracle legs (0: all cores)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
