@@ -471,6 +471,29 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
   }
 }
 
+// Key-row coordinate in the pool of page `lane` (< pages per tile) of KV tile kt0 + jt of a
+// unit with n tiles: page_table[page] << page_shift, or oob_row (the TMA fills zeros there)
+// past the unit or the table; an entry outside the pool is reported (by `report` lanes) and
+// read as oob_row. Contiguous K/V: the tile's first key row.
+template <bool PAGED>
+__device__ __forceinline__ int32_t tile_page_row(const PrefillArgs& a, int64_t kt0, int n,
+                                                 int jt, int lane, bool report) {
+  int32_t row = a.oob_row;
+  if constexpr (PAGED) {
+    const int64_t lp = (kt0 + jt) * a.pages_per_tile + lane;
+    if (jt < n && lane < a.pages_per_tile && lp < a.table_len) {
+      const int32_t e = __ldg(a.page_table + lp);
+      if (e >= 0 && e < a.num_pages)
+        row = e << a.page_shift;
+      else if (report)
+        atomicOr(&g_pa_error_flags, kFlagPage);
+    }
+  } else {
+    row = (int32_t)((kt0 + jt) * kTileKeys);
+  }
+  return row;
+}
+
 // ---------------------------------------------------------------- prefill kernel
 template <int D, bool PAGED, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -546,6 +569,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
+  // The copy warps read the page-table entries of the first two KV tiles before the set-up
+  // below, so the loads overlap it and the first copies go out right after it.
+  int32_t pre_row0 = a.oob_row, pre_row1 = a.oob_row;
+  if (warp > kMmaWarp) {
+    const bool report = warp == kMmaWarp + 1;
+    pre_row0 = tile_page_row<PAGED>(a, kt0, n, 0, lane, report);
+    pre_row1 = tile_page_row<PAGED>(a, kt0, n, 1, lane, report);
+  }
   auto bar = [&](int i) -> uint32_t { return sb + C::BAR_OFF + 8u * (uint32_t)i; };
   auto slot_addr = [&](uint32_t slot) -> uint32_t { return sb + C::RING_OFF + slot * kPanel; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF);
@@ -661,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       return r_ok;
     };
-    int32_t row_prev = a.oob_row, row_cur = fetch(0), row_next = fetch(1);
+    int32_t row_prev = a.oob_row, row_cur = pre_row0, row_next = pre_row1;
     uint32_t issued_end = 0;  // one past the last fill number this warp issued
     for (int j = 0; j <= n && ok; ++j) {
       if (j < n) {  // K tile j: panel k in fill q, one box per page (lane i: page i)

@@ -92,6 +92,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
+  // The copy warps read the page-table entries of the first two KV tiles before the set-up
+  // below, so the loads overlap it and the first copies go out right after it.
+  int32_t pre_row0 = a.oob_row, pre_row1 = a.oob_row;
+  if (warp > kMmaWarp) {
+    const bool report = warp == kMmaWarp + 1;
+    pre_row0 = tile_page_row<PAGED>(a, kt0, n, 0, lane, report);
+    pre_row1 = tile_page_row<PAGED>(a, kt0, n, 1, lane, report);
+  }
   auto bar = [&](int i) -> uint32_t { return sb + C::BAR_OFF + 8u * (uint32_t)i; };
   auto slot_addr = [&](uint32_t slot) -> uint32_t { return sb + C::RING_OFF + slot * kPanel; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF);
@@ -254,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return r_ok;
     };
     auto own_barrier = [&](uint32_t q) -> bool { return rank == 0 || tail_fill(q); };
-    int32_t row_prev = a.oob_row, row_cur = fetch(0), row_next = fetch(1);
+    int32_t row_prev = a.oob_row, row_cur = pre_row0, row_next = pre_row1;
     // Q tile: four 16 KB panels of 128/G whole tokens; both CTAs' bytes complete on rank 0's
     // barrier, which rank 0 arms for both. Rows past the piece arrive as zeros.
     if (a.q_tma && w == 0 && lane == 0) {
