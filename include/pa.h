@@ -189,7 +189,10 @@ int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes, fl
  * max_seq_len), or exactly splits_override. ws_bytes = S * batch * Hq * (D + 1) * 4 when S > 1,
  * in the layout of pa_prefill's split workspace with batch in place of R, so pa_combine
  * merges it. Returns PA_OK, PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED. Pure host code.
- * Source: the paged decode slowdown the pages measure (decode on the same paged cache).
+ * Source: generation over a long cache, where every new token reads its sequence's whole
+ * window (llama.cpp PR #27977, "qwen4exp: reduce the generation slowdown as context grows",
+ * description), on the same paged cache the prefill fills (BaseRT issue #51, "Serving impact":
+ * continuous batching implies the paged cache).
  */
 int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int page_size,
                    int batch, int64_t max_seq_len, int dtype, float scale, int splits_override,
