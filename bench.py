@@ -39,10 +39,11 @@ TRAFFIC_CAPTURE = {"workload": "c5", "sources": "815437c5a84d906b", "bytes_per_l
 
 
 def kernel_sources_hash() -> str:
-    import glob
+    """Hash of the prefill kernels' device code and of the schedule that feeds them."""
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "paged_kv_long_b200", "csrc", "*")) +
-                   [os.path.join(ROOT, "include", "pa.h")])
+    csrc = os.path.join(ROOT, "paged_kv_long_b200", "csrc")
+    files = [os.path.join(csrc, f) for f in ("pa_geometry.h", "pa_kernels.cu", "pa_plan.cpp",
+                                             "pa_schedule.h", "prefill_pair.cuh", "sm100.cuh")]
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.basename(f).encode())
