@@ -226,7 +226,8 @@ int pa_decode(const pa_plan_t* plan, const void* q, const void* k_pool, const vo
  * batching itself is the serving engine's, which the pages do not describe.
  *
  * pa_batch_plan — the balanced schedule of the batch (host only): the row blocks of all
- * sequences, longest first, cut by the wrap-around rule into at most 512 items on num_sms SMs.
+ * sequences, longest first, cut by the wrap-around rule into at most 512 items on num_sms SMs
+ * (when the cuts would not fit in 512 items, every row block is one item, longest first).
  *   q_lens     host int32 [batch], >= 0 (a sequence with 0 rows has no output rows).
  *   hist_lens  host int64 [batch], >= 0.
  *   batch      1 .. 256 sequences; at most 512 row blocks in all ((KV head, 128-row Q tile

@@ -263,7 +263,17 @@ bool build_batch(int num_sms, int head_dim, int per, int G, int Hkv, const Batch
   for (size_t i = 0; i < order.size(); ++i) order[i] = (int32_t)i;
   std::stable_sort(order.begin(), order.end(),
                    [&](int32_t x, int32_t y) { return len[x] > len[y]; });
-  return wrap_around(len, order, slots, per, head_dim, out);
+  if (wrap_around(len, order, slots, per, head_dim, out)) return true;
+  // Too many row blocks to also cut some (the item table holds 512): every row block whole,
+  // longest first, as the hardware's first-free dispatch then runs them (LPT order).
+  if (len.size() > (size_t)kMaxItems || len.empty()) return false;
+  const CostModel cm(head_dim);
+  Schedule sch;
+  sch.rows_per_block = per * kTileRows;
+  for (int32_t rb : order) sch.items.push_back(PaItem{rb, 0, (int32_t)len[rb], -1});
+  sch.makespan_us = simulate_items(sch.items, slots, cm);
+  *out = std::move(sch);
+  return true;
 }
 
 }  // namespace pa

@@ -144,8 +144,8 @@ def test_batch_schedule_covers_every_tile_once(seed):
     try:
         bp = bd.batch_plan(G * Hkv, Hkv, D, 16, q_lens, hist, "bf16", num_sms=num_sms)
     except bd.PaError as e:
-        # the item table holds 512: row blocks plus at most one cut per worker must fit
-        assert bd.STATUS[e.status] == "PA_ERR_UNSUPPORTED" and len(tiles) > 512 - num_sms // per
+        # the item table holds 512 row blocks (whole, when cuts no longer fit)
+        assert bd.STATUS[e.status] == "PA_ERR_UNSUPPORTED" and len(tiles) > 512
         return
     assert bp.plan.ctas_per_unit == per
     items = bd.batch_schedule_items(bp)
@@ -164,6 +164,24 @@ def test_batch_pairs_only_when_a_sequence_has_two_q_tiles():
     assert two.plan.ctas_per_unit == 2
     small_d = bd.batch_plan(16, 2, 128, 16, [500, 17], [900, 20], "f16", num_sms=148)
     assert small_d.plan.ctas_per_unit == 1
+
+
+def test_batch_of_many_row_blocks_keeps_them_whole():
+    """256 one-row sequences x 2 KV heads = 512 row blocks: too many to add cuts, so every row
+    block is one item, longest first."""
+    bd = _bd()
+    rng = np.random.default_rng(9)
+    hist = rng.integers(0, 20000, size=256)
+    bp = bd.batch_plan(16, 2, 128, 16, np.ones(256, dtype=np.int32), hist, "f16", num_sms=148)
+    items = bd.batch_schedule_items(bp)
+    assert len(items) == 512 and (items[:, 3] == -1).all() and bp.plan.ws_bytes == 0
+    tiles = row_block_tiles(np.ones(256, dtype=int), hist, 2, 8, 1)
+    check_items(items, tiles, TILE)
+    lens = items[:, 2] - items[:, 1]
+    assert (np.diff(lens) <= 0).all()
+    with pytest.raises(bd.PaError):   # 257 sequences: more than the sequence table holds
+        bd.batch_plan(16, 2, 128, 16, np.ones(257, dtype=np.int32), np.zeros(257), "f16",
+                      num_sms=148)
 
 
 def test_batch_schedule_balances_the_sms():
@@ -269,6 +287,20 @@ def test_gpu_batch_matches_oracle(case):
     assert bd.device_error(reset=True)[0] == 0
     U.assert_close(got, oracle_batch(sb), f"{name} (items={bp.plan.units}, "
                                           f"max parts={bp.plan.splits})")
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+def test_gpu_batch_of_256_sequences_matches_oracle():
+    """The largest batch: 256 sequences (one-row chunks and short chunks), 512 row blocks."""
+    bd = _bd()
+    rng = np.random.default_rng(51)
+    hist = rng.integers(0, 3000, size=256)
+    q_lens = np.where(np.arange(256) % 5 == 0, rng.integers(2, 16, size=256), 1)
+    sb = seq_batch(52, hist, q_lens, 16, 2, 128, 16, "bf16")
+    bp, got = run_batch(sb)
+    assert bp.plan.batch == 256 and bd.device_error(reset=True)[0] == 0
+    U.assert_close(got, oracle_batch(sb), f"256 sequences (items={bp.plan.units})")
 
 
 @pytest.mark.gpu
