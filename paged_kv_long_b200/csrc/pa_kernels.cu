@@ -1212,7 +1212,8 @@ extern "C" int pa_decode(const pa_plan_t* plan, const void* q, const void* k_poo
                          const void* v_pool, const int32_t* block_table, int table_stride,
                          const int32_t* seq_lens, int64_t num_pages, float* out, float* lse_ws,
                          uint64_t ws_bytes, pa_stream_t stream) {
-  if (!plan || plan->batch <= 0 || plan->chunk_rows != plan->batch || plan->q_tiles != 1)
+  if (!plan || plan->batch <= 0 || plan->chunk_rows != plan->batch || plan->q_tiles != 1 ||
+      plan->policy == PA_POLICY_BALANCED)  // batch plans run through pa_batch_prefill
     return PA_ERR_INVALID_ARG;
   if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !out || table_stride <= 0 ||
       num_pages <= 0)

@@ -225,6 +225,10 @@ def test_batch_abi_refuses_mixed_up_plans_and_arrays():
     st = lib.pa_batch_prefill(ctypes.byref(bp.plan), ql, hl, fake, fake, fake, fake, 1, 100,
                               fake, fake, 1 << 30, None)   # table rows too short
     assert bd.STATUS[st] == "PA_ERR_INVALID_ARG"
+    one = bd.batch_plan(16, 2, 256, 16, [1], [50], "f16", num_sms=148)  # looks like decode
+    st = lib.pa_decode(ctypes.byref(one.plan), fake, fake, fake, fake, 8, fake, 100, fake, fake,
+                       1 << 30, None)
+    assert bd.STATUS[st] == "PA_ERR_INVALID_ARG"
 
 
 @pytest.mark.parametrize("q_lens,hist,err", [
