@@ -1,0 +1,43 @@
+"""bench.py's output contract, checked on the CPU: the reference arm (the fp64 oracle timed on
+the host) prints one JSON line with the keys the driver reads, and the GPU arm's helpers are
+consistent. The GPU arm itself is run on the GPU machine."""
+import json
+import subprocess
+import sys
+
+import pytest
+
+import bench
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_prints_one_contract_line():
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "c1",
+                          "--steps", "1", "--warmup", "3", "--cpu-threads", "2"],
+                         capture_output=True, text=True, timeout=280, check=True)
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 2
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert "workload" in d["config"]
+
+
+def test_warmup_below_three_is_refused():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
+
+
+def test_traffic_capture_is_keyed_to_the_kernel_sources():
+    h = bench.kernel_sources_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+    assert set(bench.TRAFFIC_CAPTURE) == {"workload", "sources", "bytes_per_launch"}
