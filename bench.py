@@ -244,6 +244,7 @@ def time_steps(dw, steps, warmup, flush, stream, record_kernels=False):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         kev = []
+        torch.cuda.nvtx.range_push("prefill step")  # for profilers that filter on NVTX ranges
         e0.record(stream)
         for i in range(len(dw.wl.pieces)):
             if record_kernels:
@@ -258,6 +259,7 @@ def time_steps(dw, steps, warmup, flush, stream, record_kernels=False):
             else:
                 dw.run_piece(i, stream)
         e1.record(stream)
+        torch.cuda.nvtx.range_pop()
         evs.append((e0, e1, kev))
     torch.cuda.synchronize()
     for e0, e1, kev in evs:

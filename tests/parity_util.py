@@ -59,6 +59,11 @@ def run_gpu(inp: Inputs, paged=True, splits=None, policy="makespan", num_sms=Non
     from paged_kv_long_b200.runner import DeviceWorkload
     import torch
     dw = DeviceWorkload(inp, "cuda", paged=paged, splits=splits, policy=policy, num_sms=num_sms)
+    # NaN in the workspace and outputs: an entry read before it is written shows up as a
+    # non-finite output (assert_close checks finiteness)
+    dw.ws.fill_(float("nan"))
+    for o in dw.outs:
+        o.fill_(float("nan"))
     dw.run()
     torch.cuda.synchronize()
     return dw, dw.outputs_host()

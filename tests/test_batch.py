@@ -271,8 +271,13 @@ def run_batch(sb, num_sms=None):
     Hkv, PS = sb.k_pool.shape[2], sb.k_pool.shape[1]
     bp = bd.batch_plan(Hq, Hkv, D, PS, sb.q_lens, sb.hist_lens, sb.dtype, sb.scale,
                        num_sms=num_sms)
+    out = torch.full((rows, Hq, D), float("nan"), device="cuda")  # every entry must be written
+    ws = bd.workspace(bp.plan)
+    if ws is not None:
+        ws.fill_(float("nan"))
     out = bd.batch_prefill(bp, _dev(sb.q, sb.dtype), _dev(sb.k_pool, sb.dtype),
-                           _dev(sb.v_pool, sb.dtype), torch.from_numpy(sb.block_table).cuda())
+                           _dev(sb.v_pool, sb.dtype), torch.from_numpy(sb.block_table).cuda(),
+                           out, ws)
     torch.cuda.synchronize()
     return bp, out.cpu().numpy()
 

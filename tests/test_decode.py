@@ -187,9 +187,13 @@ def run_decode(db, splits=0):
     Hkv, PS = db.k_pool.shape[2], db.k_pool.shape[1]
     p = bd.decode_plan(Hq, Hkv, D, PS, B, max(1, int(db.seq_lens.max())), db.dtype,
                        scale=db.scale, splits=splits)
+    out = torch.full((B, Hq, D), float("nan"), device="cuda")  # every entry must be written
+    ws = bd.workspace(p)
+    if ws is not None:
+        ws.fill_(float("nan"))
     out = bd.decode(p, _dev(db.q, db.dtype), _dev(db.k_pool, db.dtype),
                     _dev(db.v_pool, db.dtype), torch.from_numpy(db.block_table).cuda(),
-                    torch.from_numpy(db.seq_lens).cuda())
+                    torch.from_numpy(db.seq_lens).cuda(), out, ws)
     torch.cuda.synchronize()
     return p, out.cpu().numpy()
 
