@@ -65,6 +65,21 @@ class DeviceWorkload:
         for i in range(len(self.wl.pieces)):
             self.run_piece(i, stream)
 
+    def capture(self, stream=None):
+        """The whole step (every chunk's prefill and combine) captured as one CUDA graph: the
+        plans, tensor maps and work-item tables are taken at capture (kernel parameters hold
+        them by value), so a replay launches the same work with no host-side planning."""
+        import torch
+        stream = stream or torch.cuda.Stream(self.device)
+        stream.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(stream):
+            self.run(stream)  # once outside the capture: lazy library and kernel set-up
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            self.run(torch.cuda.current_stream(self.device))
+        return graph
+
     def outputs_host(self) -> list[np.ndarray]:
         return [o.cpu().numpy() for o in self.outs]
 

@@ -273,3 +273,27 @@ def test_gpu_streamed_step_equals_the_plain_step():
     torch.cuda.synchronize()
     for i, (h, w) in enumerate(zip(houts, want)):
         assert np.array_equal(h.numpy(), w), f"piece {i}"
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("policy", ["makespan", "balanced"])
+def test_gpu_graph_replay_equals_eager(policy):
+    """A step captured as a CUDA graph (DeviceWorkload.capture) and replayed twice gives the
+    eager step's outputs bit for bit: the launches carry their plans by value."""
+    import numpy as np
+    import torch
+    wl = U.custom_workload("graph", 24, 4, 256, 64, "bf16", [(3000, 512), (3512, 300)],
+                           seed=9100)
+    inp = U.gen(wl, poison=True)
+    dw, want = U.run_gpu(inp, policy=policy)
+    graph = dw.capture()
+    for _ in range(2):
+        for o in dw.outs:
+            o.fill_(float("nan"))
+        dw.ws.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        for i, (o, w) in enumerate(zip(dw.outs, want)):
+            assert np.array_equal(o.cpu().numpy(), w), f"piece {i}"
+    assert binding.device_error(reset=True)[0] == 0
