@@ -529,7 +529,7 @@ def gpu_arm(args):
                         "launches of one step (cold L2 per launch under ncu), bytes per launch")
 
     # ---- contiguous control at the same split counts (the ratio's denominator)
-    t_contig = t_paged_pairs = last_paged = last_contig = None
+    t_contig = t_paged_pairs = last_paged = last_contig = same_bits = None
     if paged and not args.no_contiguous:
         from paged_kv_long_b200 import binding
         # the same schedule per piece as the paged run (the planner does not look at the layout)
@@ -551,6 +551,10 @@ def gpu_arm(args):
         t_contig = statistics.median(cc)
         last_paged = statistics.median(pk)
         last_contig = statistics.median(ck)
+        # verify mode: the two layouts run the same schedule on the same keys, so their outputs
+        # of the last step must be the same bits
+        torch.cuda.synchronize()
+        same_bits = all(torch.equal(a_, b_) for a_, b_ in zip(dw.outs, dwc.outs))
         del dwc
 
     # ---- KV append, the step before prefill (its own HBM roofline)
@@ -610,6 +614,7 @@ def gpu_arm(args):
         "paged_contiguous_ratio_last_chunk": (last_contig / last_paged) if t_contig else None,
         "contiguous_ms_per_step": t_contig,
         "ratio_method": "median of alternating paged / contiguous steps (L2 flushed before each)",
+        "paged_contiguous_outputs_identical": same_bits,
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": traffic,
                      "traffic_source": traffic_note,
