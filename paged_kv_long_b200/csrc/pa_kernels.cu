@@ -860,11 +860,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
   const float inv = W > 0.f ? 1.f / W : 0.f;
-  for (int d0 = lane * 4; d0 < D; d0 += 128) {
+  // Every lane runs the same column passes and takes part in every shuffle (at D = 64 only
+  // lanes 0-15 own columns, but the weights of splits 16-31 sit in lanes 16-31).
+  for (int d0 = lane * 4; d0 < D + lane * 4; d0 += 128) {
+    const bool mine = d0 < D;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int sp = 0; sp < S; ++sp) {
       const float ws = __shfl_sync(0xffffffffu, wt, sp);
-      if (ws != 0.f) {
+      if (mine && ws != 0.f) {
         const float4 o = *reinterpret_cast<const float4*>(ws_o + ((int64_t)sp * RH + w) * D + d0);
         acc.x = fmaf(ws, o.x, acc.x);
         acc.y = fmaf(ws, o.y, acc.y);
@@ -872,8 +875,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         acc.w = fmaf(ws, o.w, acc.w);
       }
     }
-    *reinterpret_cast<float4*>(out + w * D + d0) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (mine)
+      *reinterpret_cast<float4*>(out + w * D + d0) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
 }
 
@@ -920,11 +924,13 @@ __global__ void __launch_bounds__(256) combine_blocks_kernel(
   for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
   const float inv = W > 0.f ? 1.f / W : 0.f;
   float* dst = out + (tok * Hq + head) * (int64_t)D;
-  for (int d0 = lane * 4; d0 < D; d0 += 128) {
+  // every lane joins every shuffle (see combine_kernel)
+  for (int d0 = lane * 4; d0 < D + lane * 4; d0 += 128) {
+    const bool mine = d0 < D;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int sp = 0; sp < b.nparts; ++sp) {
       const float ws = __shfl_sync(0xffffffffu, wt, sp);
-      if (ws != 0.f) {
+      if (mine && ws != 0.f) {
         const float4 o =
             *reinterpret_cast<const float4*>(ws_o + (row0 + (int64_t)sp * rows_per_block) * D + d0);
         acc.x = fmaf(ws, o.x, acc.x);
@@ -933,8 +939,9 @@ __global__ void __launch_bounds__(256) combine_blocks_kernel(
         acc.w = fmaf(ws, o.w, acc.w);
       }
     }
-    *reinterpret_cast<float4*>(dst + d0) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (mine)
+      *reinterpret_cast<float4*>(dst + d0) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
 }
 

@@ -171,6 +171,7 @@ CASES = [
     ("d128_empty_s1", [0, 3, 1], 8, 8, 128, 16, "f16", 1),
     ("d64_g16", [700, 64, 1500], 32, 2, 64, 128, "f16", 0),
     ("d64_g1", [33, 800], 4, 4, 64, 16, "bf16", 4),
+    ("d64_24_splits", [3000, 5, 130], 8, 1, 64, 16, "f16", 24),
 ]
 
 

@@ -59,6 +59,9 @@ RAGGED = [
     (12, 3, 64, 64, "f16", [(0, 1)], 1),
     (24, 4, 256, 64, "bf16", [(4000, 1)], 32),
     (16, 2, 256, 16, "f16", [(10, 16)], 8),      # more splits than KV tiles: empty splits
+    # head dim 64 merges more than 16 splits: lanes 16-31 own no columns but hold weights
+    (8, 1, 64, 128, "bf16", [(0, 1)], 32),
+    (8, 2, 64, 16, "bf16", [(0, 369)], 17),
 ]
 
 
