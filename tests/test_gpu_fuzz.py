@@ -3,8 +3,11 @@ sampled (row, head) pairs (first and last rows, Q-tile edges, random rest) with 
 beyond the keys, workspaces and outputs, so a wrong key, a missed write or a stale partial fails.
 
 Single pieces: head dim, GQA group, page size, dtype, history (0 .. 40K, often off a page or
-tile edge), chunk rows (1 .. 1,500), policy (planner, balanced, forced splits 1 .. 32).
+tile edge), chunk rows (1 .. 1,500), policy (planner, balanced, forced splits 1 .. 32), paged
+or contiguous K/V.
 Batches: 1 .. 12 sequences of random histories and rows, one-row (decode) batches included.
+Decode (pa_decode, device-side lengths): 1 .. 40 sequences of 0 .. 20,000 keys, split counts
+from the planner or forced (1 .. 32).
 """
 import math
 
@@ -15,8 +18,9 @@ from oracle import oracle
 from tests.conftest import cuda_available
 from tests import parity_util as U
 
-N_PIECE = 24
-N_BATCH = 10
+N_PIECE = 48
+N_BATCH = 20
+N_DECODE = 12
 
 
 def piece_case(seed):
@@ -31,7 +35,8 @@ def piece_case(seed):
     mode = str(rng.choice(["planner", "balanced", "forced"]))
     S = int(rng.choice([1, 2, 3, 5, 8, 17, 32])) if mode == "forced" else None
     num_sms = int(rng.choice([148, 148, 37, 9]))
-    return D, Hkv, G, PS, dtype, H, R, mode, S, num_sms
+    paged = bool(seed % 5 != 4)  # every fifth piece reads contiguous K/V
+    return D, Hkv, G, PS, dtype, H, R, mode, S, num_sms, paged
 
 
 @pytest.mark.gpu
@@ -39,16 +44,18 @@ def piece_case(seed):
 @pytest.mark.parametrize("seed", range(N_PIECE))
 def test_gpu_fuzz_piece(seed):
     from paged_kv_long_b200 import binding
-    D, Hkv, G, PS, dtype, H, R, mode, S, num_sms = piece_case(seed)
-    name = f"fuzz{seed}: D{D} Hkv{Hkv} G{G} PS{PS} {dtype} H{H} R{R} {mode} S={S} sms{num_sms}"
+    D, Hkv, G, PS, dtype, H, R, mode, S, num_sms, paged = piece_case(seed)
+    name = (f"fuzz{seed}: D{D} Hkv{Hkv} G{G} PS{PS} {dtype} H{H} R{R} {mode} S={S} "
+            f"sms{num_sms} {'paged' if paged else 'contiguous'}")
     wl = U.custom_workload(name, Hkv * G, Hkv, D, PS, dtype, [(H, R)], seed=20000 + 10 * seed,
                            splits=S or 0)
     inp = U.gen(wl, poison=True)
     binding.device_error(reset=True)
     policy = "balanced" if mode == "balanced" else "makespan"
-    dw, outs = U.run_gpu(inp, splits=S if S else 0, policy=policy, num_sms=num_sms)
+    dw, outs = U.run_gpu(inp, paged=paged, splits=S if S else 0, policy=policy,
+                         num_sms=num_sms)
     assert binding.device_error(reset=True)[0] == 0, name
-    U.check_sampled(inp, outs, n=40, what=name)
+    U.check_sampled(inp, outs, n=40, paged=paged, what=name)
 
 
 def batch_case(seed):
@@ -111,3 +118,58 @@ def test_gpu_fuzz_batch(seed):
         sel_r, sel_h = U.sample_pairs(r, Hq, 12, 40000 + seed * 64 + b, G)
         ref, _ = oracle.attend(pb, sel_r, sel_h)
         U.assert_close(got[r0s[b] + sel_r, sel_h], ref, f"{name} sequence {b} (H={h}, R={r})")
+
+
+def decode_case(seed):
+    rng = np.random.default_rng(9000 + seed)
+    D = int(rng.choice([64, 128, 256]))
+    Hkv = int(rng.choice([1, 2, 8]))
+    G = int(rng.choice([1, 4, 8, 16]))
+    PS = int(rng.choice([16, 32, 128]))
+    dtype = str(rng.choice(["f16", "bf16"]))
+    B = int(rng.integers(1, 41))
+    lens = rng.integers(0, 20000, size=B)
+    lens[rng.integers(0, B)] = int(rng.choice([0, 1, 128, 129]))
+    S = int(rng.choice([0, 0, 1, 7, 19, 32]))
+    return D, Hkv, G, PS, dtype, lens, S
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("seed", range(N_DECODE))
+def test_gpu_fuzz_decode(seed):
+    import torch
+    from paged_kv_long_b200 import binding
+    from paged_kv_long_b200.inputs import decode_batch
+    D, Hkv, G, PS, dtype, lens, S = decode_case(seed)
+    Hq = Hkv * G
+    name = f"decode fuzz{seed}: D{D} Hkv{Hkv} G{G} PS{PS} {dtype} B{len(lens)} S={S}"
+    db = decode_batch(50000 + seed, lens, Hq, Hkv, D, PS, dtype)
+    p = binding.decode_plan(Hq, Hkv, D, PS, len(lens), max(1, int(lens.max())), dtype, splits=S)
+    binding.device_error(reset=True)
+
+    def dev(bits):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda()
+        return t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+
+    out = torch.full((len(lens), Hq, D), float("nan"), device="cuda")
+    ws = binding.workspace(p)
+    if ws is not None:
+        ws.fill_(float("nan"))
+    binding.decode(p, dev(db.q), dev(db.k_pool), dev(db.v_pool),
+                   torch.from_numpy(db.block_table).cuda(), torch.from_numpy(db.seq_lens).cuda(),
+                   out, ws)
+    torch.cuda.synchronize()
+    assert binding.device_error(reset=True)[0] == 0, name
+    got = out.cpu().numpy()
+    heads = np.random.default_rng(seed).integers(0, Hq, size=len(lens)).astype(np.int32)
+    for b, n in enumerate(lens):
+        n = int(n)
+        if n == 0:
+            assert (got[b] == 0).all(), f"{name}: sequence {b} has no key, output must be 0"
+            continue
+        pb = oracle.Problem(q=db.q[b:b + 1], k=db.k_pool, v=db.v_pool, hist_len=n - 1,
+                            dtype=dtype, page_table=db.block_table[b, :math.ceil(n / PS)])
+        hs = np.array([0, Hq - 1, heads[b]], dtype=np.int32)
+        ref, _ = oracle.attend(pb, np.zeros(3, dtype=np.int64), hs)
+        U.assert_close(got[b, hs], ref, f"{name} sequence {b} ({n} keys)")
