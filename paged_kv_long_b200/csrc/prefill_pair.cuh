@@ -356,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         PA_UNIT_ONLY(const long long c0 = clock64();)
         const bool r = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
         PA_UNIT_ONLY(*w_sel += clock64() - c0;)
+        PA_TRACE_ONLY(tlog(6, tln_w, 12, round * NSLOT + slot);)
         return r;
       };
       auto advance = [&]() {
