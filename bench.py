@@ -35,7 +35,7 @@ L2_FLUSH_BYTES = 512 << 20
 # (profiles/prefill_pair_kernel_c5_traffic.md: dram__bytes_read.sum + dram__bytes_write.sum
 # over the timed step's 16 launches / 16). It stands for the kernel whose sources hash to
 # `sources`; after any change to them the bench reports null until it is captured again.
-TRAFFIC_CAPTURE = {"workload": "c5", "sources": "5c4f67523becf5f6", "bytes_per_launch": 107.39e6}
+TRAFFIC_CAPTURE = {"workload": "c5", "sources": "8312d6da92add253", "bytes_per_launch": 106.76e6}
 
 
 def kernel_sources_hash() -> str:
