@@ -173,3 +173,41 @@ def test_gpu_fuzz_decode(seed):
         hs = np.array([0, Hq - 1, heads[b]], dtype=np.int32)
         ref, _ = oracle.attend(pb, np.zeros(3, dtype=np.int64), hs)
         U.assert_close(got[b, hs], ref, f"{name} sequence {b} ({n} keys)")
+
+
+N_APPEND = 8
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("seed", range(N_APPEND))
+def test_gpu_fuzz_kv_append(seed):
+    """pa_kv_append on random shapes and positions, bit for bit against the append oracle."""
+    import torch
+    from oracle.kv_append import kv_append as oracle_append
+    from paged_kv_long_b200 import binding
+    rng = np.random.default_rng(60000 + seed)
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    D = int(rng.choice([64, 128, 256]))
+    PS = int(rng.choice([16, 32, 64, 128]))
+    H = int(rng.choice([0, int(rng.integers(1, 5000))]))
+    R = int(rng.choice([1, int(rng.integers(2, 3000))]))
+    pages = math.ceil((H + R) / PS)
+    num_pages = pages + int(rng.integers(0, 9))
+    pool = rng.integers(0, 1 << 16, size=(num_pages, PS, Hkv, D), dtype=np.uint16)
+    new = rng.integers(0, 1 << 16, size=(R, Hkv, D), dtype=np.uint16)
+    table = rng.permutation(num_pages)[:pages].astype(np.int32)
+    want, bad = oracle_append(pool, new, table, H)
+    assert bad == 0
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(
+            torch.bfloat16)
+
+    kp, vp = dev(pool), dev(pool.copy())
+    binding.device_error(reset=True)
+    binding.kv_append(dev(new), dev(new), kp, vp, torch.from_numpy(table).cuda(), H)
+    torch.cuda.synchronize()
+    assert binding.device_error(reset=True)[0] == 0
+    for t in (kp, vp):
+        assert np.array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16), want)

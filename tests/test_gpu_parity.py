@@ -107,6 +107,8 @@ BALANCED = [
     (6, 2, 128, 32, "f16", [(1500, 131)], 6),
     (4, 1, 64, 16, "bf16", [(2500, 99)], 3),
     (4, 1, 64, 16, "f16", [(9000, 30)], 4),
+    # one long row block over 148 SMs at head dim 64: more than 16 parts to merge
+    (4, 1, 64, 16, "f16", [(30000, 20)], 148),
 ]
 
 
