@@ -35,20 +35,25 @@ L2_FLUSH_BYTES = 512 << 20
 # (profiles/prefill_pair_kernel_c5_traffic.md: dram__bytes_read.sum + dram__bytes_write.sum
 # over the timed step's 16 launches / 16). It stands for the kernel whose sources hash to
 # `sources`; after any change to them the bench reports null until it is captured again.
-TRAFFIC_CAPTURE = {"workload": "c5", "sources": "8312d6da92add253", "bytes_per_launch": 106.76e6}
+TRAFFIC_CAPTURE = {"workload": "c5", "sources": "1b256855e328955e", "bytes_per_launch": 106.76e6}
 
 
 def kernel_sources_hash() -> str:
-    """Hash of the prefill kernels' device code and of the schedule that feeds them."""
+    """Hash of the prefill kernels' device code and of the schedule that feeds them, comments
+    and blank lines left out (a comment edit does not change the kernel)."""
     import hashlib
+    import re
     csrc = os.path.join(ROOT, "paged_kv_long_b200", "csrc")
     files = [os.path.join(csrc, f) for f in ("pa_geometry.h", "pa_kernels.cu", "pa_plan.cpp",
                                              "pa_schedule.h", "prefill_pair.cuh", "sm100.cuh")]
     h = hashlib.sha256()
     for f in files:
+        with open(f) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        code = [ln.split("//")[0].rstrip() for ln in text.splitlines()]
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        h.update("\n".join(ln for ln in code if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

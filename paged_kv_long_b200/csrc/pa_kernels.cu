@@ -1,15 +1,17 @@
 // pa_kernels.cu — sm_100a kernels of libpa and their C-ABI entry points.
 //
-// prefill_kernel: one CTA per (KV head, packed Q tile, history split) unit.
+// prefill_kernel: one CTA per unit — (KV head, packed Q tile, history split) for uniform splits,
+//   a work item (a run of a row block's KV tiles) for balanced plans, (sequence, KV head, split)
+//   for batched decode.
 //   The operation is prefill attention of a query chunk against a long history read through
 //   a paged KV cache (BaseRT issue #51, "Results"), with the history of a piece cut into
 //   splits whose partials a reduce merges (splash PR #33, "What changed"). The B200 design:
-//   * warp 4 (producer) reads the page table and issues TMA boxes into a ring of 16 KB,
+//   * warps 5-7 (copy warps) read the page table and issue TMA boxes into a ring of 16 KB,
 //     128-byte-swizzled shared-memory panels: K as one box per (page, 64-wide D panel), V as
-//     one box per (page, half of D);
-//   * warp 5 (MMA) issues tcgen05.mma: S = Q K^T into one of two tensor-memory S buffers
-//     (Q and K from shared memory), then O += P V with P read from tensor memory where the
-//     softmax wrote it over its own S buffer (fp32 accumulation in tensor memory);
+//     boxes of up to one page covering all of D;
+//   * warp 4 (MMA; one lane) issues tcgen05.mma: S = Q K^T into one of two tensor-memory S
+//     buffers (Q and K from shared memory), then O += P V with P read from tensor memory where
+//     the softmax wrote it over its own S buffer (fp32 accumulation in tensor memory);
 //   * warps 0-3 (softmax, one thread per packed Q row = tensor-memory lane) load the GQA-
 //     packed Q tile, read S with tcgen05.ld, apply the causal mask by select, keep the
 //     running max and sum (rescaling O only when the max grows by more than 2^8), write P
@@ -17,8 +19,11 @@
 //     split partial and its base-2 log-sum-exp.
 //   Every wait is bounded: on expiry the kernel sets the timeout bit, abandons its work,
 //   waits for its own copies and MMAs in flight, frees tensor memory and exits.
+// prefill_pair_kernel (prefill_pair.cuh): head dim 256 on CTA pairs (cta_group::2, M = 256).
 // combine_kernel: one warp per (row, head) merges the S partials with a log-sum-exp
-//   weighting (the "reduce" of splash PR #33).
+//   weighting (the "reduce" of splash PR #33); combine_blocks_kernel does the same for the
+//   cut row blocks of balanced plans.
+// kv_append_kernel (kv_append.cuh): a chunk's K/V rows into their pages.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
