@@ -11,8 +11,8 @@
  *   section "Reproduction"/"Scaling characteristic": prefill attention that reads its K/V
  *   through a paged cache must give what the contiguous cache gives.
  *   "perf: scale prefill attention splits with GPU cores on Apple7/8" (splash PR #33),
- *   section "Testing": the split kernel is checked "against a CPU reference"; splitting the
- *   history changes only rounding.
+ *   section "Testing": the split kernel is verified by comparison with a CPU implementation;
+ *   splitting the history changes only rounding.
  *   Shapes: 24 Q / 4 KV heads, D256 ("KVarN V-store per-call latency ..." issue #163, Setup);
  *   16 Q / 2 KV heads, head_dim 256 (BaseRT issue #51, "Model provenance").
  *
