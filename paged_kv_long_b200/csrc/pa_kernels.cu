@@ -122,6 +122,31 @@ __device__ __forceinline__ int32_t batch_rebase(PrefillArgs& a, const ItemTable&
   return rb - sq.rb0;
 }
 
+// Device-length decode: block r·Hkv·S .. of the grid runs the sequence of rank r, where the rank
+// orders the sequences by length, longest first (ties by index). The block scheduler hands out
+// blocks in index order as SMs free up, so the units of the longest sequences start first and
+// the short ones fill the end (longest-processing-time-first list scheduling). A bijection of
+// 0 .. B-1 whatever the lengths hold. Every thread of the block takes part (two block barriers);
+// `scratch` is B + 1 words of shared memory that no copy writes yet.
+constexpr int kRankedSeqsMax = 256;  // longer batches keep the sequence order
+
+__device__ __noinline__ int seq_of_rank(const int32_t* lens, int B, int r, int32_t* scratch) {
+  for (int i = threadIdx.x; i < B; i += blockDim.x) scratch[i] = __ldg(lens + i);
+  if (threadIdx.x == 0) scratch[B] = r;
+  __syncthreads();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int32_t lb = scratch[b];
+    int rank = 0;
+    for (int c = 0; c < B; ++c) {
+      const int32_t lc = scratch[c];
+      rank += (lc > lb) | ((lc == lb) & (c < b));
+    }
+    if (rank == r) scratch[B] = b;  // exactly one b has rank r
+  }
+  __syncthreads();
+  return scratch[B];
+}
+
 // Shared-memory layout. The ring holds 16 KB slots, filled and consumed in the order K0, K1,
 // V0, K2, V1, ..., V_{n-1}; every K or V tile takes NP consecutive slots (mod NSLOT). A K
 // tile is one 64-wide D panel per slot (128 keys x 128 B, the K-major B operand of Q K^T),
@@ -526,7 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (a.batch > 0) {
     // one new token of sequence b: keys 0 .. len-1 (its own included), all visible
     const int64_t per_seq = (int64_t)a.Hkv * a.splits;
-    const int64_t b = blockIdx.x / per_seq, rem = blockIdx.x % per_seq;
+    const int64_t rem = blockIdx.x % per_seq;
+    int64_t b = blockIdx.x / per_seq;
+    if (a.batch <= kRankedSeqsMax)
+      b = seq_of_rank(a.seq_lens, a.batch, (int)b,
+                      reinterpret_cast<int32_t*>(smem + C::RING_OFF));
     g = (int)(rem / a.splits);
     s = (int)(rem % a.splits);
     qt = 0;

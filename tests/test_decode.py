@@ -232,6 +232,25 @@ def test_gpu_decode_long_batch_sampled():
 
 @pytest.mark.gpu
 @pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("B", [255, 256, 257])
+def test_gpu_decode_longest_first_dispatch_edges(B):
+    """Blocks go to sequences longest first (ties by index) up to 256 sequences, in sequence
+    order beyond: both sides of that edge, with runs of equal lengths and empty sequences,
+    every output against the oracle."""
+    rng = np.random.default_rng(800 + B)
+    lens = rng.integers(0, 400, size=B)
+    lens[::7] = 129          # a run of ties across the batch
+    lens[3::11] = 0
+    db = decode_batch(801 + B, lens, 8, 2, 64, 16, "f16")
+    p, got = run_decode(db, splits=3)
+    assert _binding().device_error(reset=True)[0] == 0
+    empty = db.seq_lens == 0
+    assert (got[empty] == 0).all()
+    U.assert_close(got[~empty], oracle_decode(db)[~empty], f"B={B} (S={p.splits})")
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
 def test_gpu_decode_length_past_table_is_reported():
     import torch
     bd = _binding()
