@@ -246,6 +246,24 @@ def test_c5_full_size_sampled_paged_equals_contiguous():
         assert np.array_equal(a, b)
 
 
+# ------------------------------------------------------------------ beyond the five workloads
+@pytest.mark.parametrize("case", [
+    # name, Hq, Hkv, D, PS, dtype, (H, R): histories of 2^20 and 2^22 keys plus a ragged tail,
+    # 8,000-33,000 KV tiles per row block and 5.2 M pool rows (the largest coordinates here)
+    ("million_d256", 8, 1, 256, 128, "bf16", (1_048_576 + 77, 200)),
+    ("four_million_d64", 4, 1, 64, 64, "f16", (4_194_304 + 1_000, 130)),
+], ids=lambda c: c[0])
+def test_longest_histories_sampled(case):
+    name, Hq, Hkv, D, PS, dt, piece = case
+    wl = U.custom_workload(name, Hq, Hkv, D, PS, dt, [piece], seed=4242)
+    inp = U.gen(wl)
+    _, o_plan = U.run_gpu(inp)                          # the planner (balanced items)
+    U.check_sampled(inp, o_plan, n=24, what=f"{name} planned")
+    _, o_32 = U.run_gpu(inp, splits=32)                 # the most uniform splits
+    U.check_sampled(inp, o_32, n=12, what=f"{name} S=32")
+    assert np.abs(o_plan[0].astype(np.float64) - o_32[0]).max() <= 2.0 ** -10
+
+
 @pytest.mark.gpu
 @pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
 def test_gpu_streamed_step_equals_the_plain_step():
