@@ -251,6 +251,53 @@ def test_gpu_decode_longest_first_dispatch_edges(B):
 
 @pytest.mark.gpu
 @pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
+def test_gpu_decode_graph_replay_follows_device_lengths():
+    """pa_decode (+ pa_combine) captured once in a CUDA graph, then replayed while the lengths
+    and the query tokens change in place on the device: a step that appends one token to every
+    sequence, then lengths redrawn so that the longest-first order changes. Each replay equals
+    the oracle at that step's lengths."""
+    import dataclasses
+    import torch
+    from paged_kv_long_b200.inputs import to_bits
+    bd = _binding()
+    B, Hq, Hkv, D, PS, dt = 12, 16, 2, 128, 16, "bf16"
+    rng = np.random.default_rng(91)
+    lens0 = rng.integers(100, 3000, size=B)
+    cap = lens0 + 600                                   # pages for the longest lengths below
+    db = decode_batch(92, cap, Hq, Hkv, D, PS, dt)
+    p = bd.decode_plan(Hq, Hkv, D, PS, B, int(cap.max()), dt)
+    assert p.splits > 1                                 # the combine is in the graph too
+    q = _dev(db.q, dt).clone()
+    kp, vp = _dev(db.k_pool, dt), _dev(db.v_pool, dt)
+    tab = torch.from_numpy(db.block_table).cuda()
+    sl = torch.from_numpy(lens0.astype(np.int32)).cuda()
+    out = torch.zeros((B, Hq, D), device="cuda")
+    ws = bd.workspace(p)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        bd.decode(p, q, kp, vp, tab, sl, out, ws, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        bd.decode(p, q, kp, vp, tab, sl, out, ws, stream=s)
+    bd.device_error(reset=True)
+    steps = [lens0, lens0 + 1, cap - rng.integers(0, 600, size=B)]
+    for i, lens in enumerate(steps):
+        q_bits = to_bits(rng.standard_normal((B, Hq, D), dtype=np.float32), dt)
+        q.copy_(_dev(q_bits, dt))
+        sl.copy_(torch.from_numpy(lens.astype(np.int32)))
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert bd.device_error(reset=True)[0] == 0
+        ref = oracle_decode(dataclasses.replace(db, q=q_bits, seq_lens=lens.astype(np.int32)))
+        U.assert_close(out.cpu().numpy(), ref, f"graph replay {i} (S={p.splits})")
+    del g
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
 def test_gpu_decode_length_past_table_is_reported():
     import torch
     bd = _binding()
