@@ -875,9 +875,71 @@ __global__ void __launch_bounds__(kThreads, 1)
 #include "prefill_pair.cuh"
 #include "kv_append.cuh"
 
-// ---------------------------------------------------------------- combine kernel
-// One warp per (row, head): lanes hold the S <= 32 split LSEs, the warp reduces max and sum
-// by shuffles, then each lane accumulates 4 output columns per step.
+// ---------------------------------------------------------------- combine kernels
+// The merge of one output row (one warp): part p's partial row is at o + p * o_stride (D fp32,
+// already divided by its own sum) and its base-2 LSE at lse + p * lse_stride, p < np <= 32.
+// Lane p holds LSE p; shuffles give M = max and W = sum of 2^(lse_p - M); the row is
+// sum_p 2^(lse_p - M) O_p / W, parts of weight 0 skipped, multiply-adds in part order. Loads
+// go out four parts at a time, both 128-column passes together, and the first four are issued
+// before the weights are known: one memory latency per four parts, not one per part and pass.
+// Every lane takes part in every shuffle (at D = 64 only lanes 0-15 own columns, but the
+// weights of parts 16-31 sit in lanes 16-31).
+template <int NPASS>  // 128-column passes: 1 for D = 64 and 128, 2 for D = 256
+__device__ __forceinline__ void merge_row(const float* __restrict__ o, int64_t o_stride,
+                                          const float* __restrict__ lse_p, int64_t lse_stride,
+                                          int np, int D, float* __restrict__ dst, int lane) {
+  constexpr int kGroup = 4;
+  const float lse = lane < np ? lse_p[(int64_t)lane * lse_stride] : -INFINITY;
+  float4 v[kGroup][NPASS];
+  auto load_group = [&](int p0) {
+#pragma unroll
+    for (int k = 0; k < kGroup; ++k)
+#pragma unroll
+      for (int ps = 0; ps < NPASS; ++ps) {
+        const int d0 = lane * 4 + 128 * ps;
+        v[k][ps] = (p0 + k < np && d0 < D)
+                       ? *reinterpret_cast<const float4*>(o + (int64_t)(p0 + k) * o_stride + d0)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+  };
+  load_group(0);
+  float M = lse;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float wt = (lse == -INFINITY) ? 0.f : exp2f(lse - M);
+  float W = wt;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  float4 acc[NPASS];
+#pragma unroll
+  for (int ps = 0; ps < NPASS; ++ps) acc[ps] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p0 = 0; p0 < np; p0 += kGroup) {  // np is the same in every lane
+    if (p0 > 0) load_group(p0);
+#pragma unroll
+    for (int k = 0; k < kGroup; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wt, (p0 + k) & 31);
+      if (p0 + k < np && w != 0.f) {
+#pragma unroll
+        for (int ps = 0; ps < NPASS; ++ps) {
+          acc[ps].x = fmaf(w, v[k][ps].x, acc[ps].x);
+          acc[ps].y = fmaf(w, v[k][ps].y, acc[ps].y);
+          acc[ps].z = fmaf(w, v[k][ps].z, acc[ps].z);
+          acc[ps].w = fmaf(w, v[k][ps].w, acc[ps].w);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int ps = 0; ps < NPASS; ++ps) {
+    const int d0 = lane * 4 + 128 * ps;
+    if (d0 < D)
+      *reinterpret_cast<float4*>(dst + d0) = make_float4(acc[ps].x * inv, acc[ps].y * inv,
+                                                         acc[ps].z * inv, acc[ps].w * inv);
+  }
+}
+
+// Uniform splits: one warp per (row, head) merges its S <= 32 split partials into out.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ ws_o,
                                                       const float* __restrict__ ws_lse,
                                                       float* __restrict__ out, int S, int64_t RH,
@@ -885,34 +947,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (w >= RH) return;
   const int lane = threadIdx.x & 31;
-  const float lse = lane < S ? ws_lse[(int64_t)lane * RH + w] : -INFINITY;
-  float M = lse;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float wt = (lse == -INFINITY) ? 0.f : exp2f(lse - M);
-  float W = wt;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
-  const float inv = W > 0.f ? 1.f / W : 0.f;
-  // Every lane runs the same column passes and takes part in every shuffle (at D = 64 only
-  // lanes 0-15 own columns, but the weights of splits 16-31 sit in lanes 16-31).
-  for (int d0 = lane * 4; d0 < D + lane * 4; d0 += 128) {
-    const bool mine = d0 < D;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < S; ++sp) {
-      const float ws = __shfl_sync(0xffffffffu, wt, sp);
-      if (mine && ws != 0.f) {
-        const float4 o = *reinterpret_cast<const float4*>(ws_o + ((int64_t)sp * RH + w) * D + d0);
-        acc.x = fmaf(ws, o.x, acc.x);
-        acc.y = fmaf(ws, o.y, acc.y);
-        acc.z = fmaf(ws, o.z, acc.z);
-        acc.w = fmaf(ws, o.w, acc.w);
-      }
-    }
-    if (mine)
-      *reinterpret_cast<float4*>(out + w * D + d0) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  }
+  if (D == 256)
+    merge_row<2>(ws_o + w * D, RH * D, ws_lse + w, RH, S, D, out + w * D, lane);
+  else
+    merge_row<1>(ws_o + w * D, RH * D, ws_lse + w, RH, S, D, out + w * D, lane);
 }
 
 // Balanced plans: one warp per packed row of a cut row block merges that row's parts (workspace
@@ -948,35 +986,12 @@ __global__ void __launch_bounds__(256) combine_blocks_kernel(
   if (tok >= R) return;
   const int head = g * G + (int)(grow % G);
   const int64_t row0 = (int64_t)b.first_slot * rows_per_block + lr;  // part p: row0 + p * rpb
-  const float lse = lane < b.nparts ? ws_lse[row0 + (int64_t)lane * rows_per_block] : -INFINITY;
-  float M = lse;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float wt = (lse == -INFINITY) ? 0.f : exp2f(lse - M);
-  float W = wt;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
-  const float inv = W > 0.f ? 1.f / W : 0.f;
   float* dst = out + (tok * Hq + head) * (int64_t)D;
-  // every lane joins every shuffle (see combine_kernel)
-  for (int d0 = lane * 4; d0 < D + lane * 4; d0 += 128) {
-    const bool mine = d0 < D;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < b.nparts; ++sp) {
-      const float ws = __shfl_sync(0xffffffffu, wt, sp);
-      if (mine && ws != 0.f) {
-        const float4 o =
-            *reinterpret_cast<const float4*>(ws_o + (row0 + (int64_t)sp * rows_per_block) * D + d0);
-        acc.x = fmaf(ws, o.x, acc.x);
-        acc.y = fmaf(ws, o.y, acc.y);
-        acc.z = fmaf(ws, o.z, acc.z);
-        acc.w = fmaf(ws, o.w, acc.w);
-      }
-    }
-    if (mine)
-      *reinterpret_cast<float4*>(dst + d0) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  }
+  const int64_t rpb = rows_per_block;
+  if (D == 256)
+    merge_row<2>(ws_o + row0 * D, rpb * D, ws_lse + row0, rpb, b.nparts, D, dst, lane);
+  else
+    merge_row<1>(ws_o + row0 * D, rpb * D, ws_lse + row0, rpb, b.nparts, D, dst, lane);
 }
 
 // ---------------------------------------------------------------- timeout self-test
