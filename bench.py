@@ -641,7 +641,13 @@ def gpu_arm(args):
                      "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": traffic,
                      "traffic_source": traffic_note,
                      "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                     # the same kernel against the measured seconds-long, power-capped GEMM rate
+                     "frac_of_sustained_peak": kern_tflops / peaks["bf16_tflops_sustained"],
                      "step_frac_of_roofline": t_roof / (t_step / 1e3),
+                     # the step split: the prefill launches' summed event time, and the rest
+                     # (the merges of split pieces and the gaps between launches)
+                     "kernel_ms_per_step": kern_total_ms,
+                     "outside_kernel_ms_per_step": t_step - kern_total_ms,
                      "kernel": "prefill_pair_kernel (pa_prefill, head dim 256)" if wl.head_dim == 256 else "prefill_kernel (pa_prefill)",
                      "algorithmic_flops_per_step": flops},
         "e2e": e2e,
