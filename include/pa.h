@@ -210,9 +210,10 @@ int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int
  *   lse_ws       workspace of plan->ws_bytes when S > 1; then call pa_combine (same plan).
  * Returns PA_OK, PA_ERR_INVALID_ARG, PA_ERR_WORKSPACE or PA_ERR_CUDA; bad page entries and
  * wait timeouts are reported by pa_device_error.
- * For batch <= 256 the kernel reads seq_lens first and starts the units of the longest
- * sequences first (ties in sequence order), so the short ones fill the end of the launch;
- * larger batches run in sequence order. The order changes timing only, never the results.
+ * The kernel reads seq_lens first and starts the units of the longest sequences first, so the
+ * short ones fill the end of the launch: for batch <= 256 by exact length (ties in sequence
+ * order), for larger batches by length class floor(log2(ceil(len / 128))) (sequence order
+ * within a class). The order changes timing only, never the results.
  */
 int pa_decode(const pa_plan_t* plan, const void* q, const void* k_pool, const void* v_pool,
               const int32_t* block_table, int table_stride, const int32_t* seq_lens,

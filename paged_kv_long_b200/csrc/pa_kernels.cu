@@ -128,7 +128,7 @@ __device__ __forceinline__ int32_t batch_rebase(PrefillArgs& a, const ItemTable&
 // the short ones fill the end (longest-processing-time-first list scheduling). A bijection of
 // 0 .. B-1 whatever the lengths hold. Every thread of the block takes part (two block barriers);
 // `scratch` is B + 1 words of shared memory that no copy writes yet.
-constexpr int kRankedSeqsMax = 256;  // longer batches keep the sequence order
+constexpr int kRankedSeqsMax = 256;  // longer batches: by length class (seq_of_class_rank)
 
 __device__ __noinline__ int seq_of_rank(const int32_t* lens, int B, int r, int32_t* scratch) {
   for (int i = threadIdx.x; i < B; i += blockDim.x) scratch[i] = __ldg(lens + i);
@@ -145,6 +145,65 @@ __device__ __noinline__ int seq_of_rank(const int32_t* lens, int B, int r, int32
   }
   __syncthreads();
   return scratch[B];
+}
+
+// Longer batches: the same longest-first rule at the granularity of a factor of two. Sequences
+// are ordered by length class floor(log2(KV tiles)) (a sequence with no key counts as one
+// tile), the longest class first, sequence order within a class; O(B / threads) per block.
+// The class of rank r comes from per-class counts; its member of index r - (the counts of the
+// longer classes) from a block scan of per-thread counts over contiguous runs of sequences.
+// A bijection of 0 .. B-1. Every thread of the block takes part (five block barriers);
+// `scratch` is 67 words of shared memory that no copy writes yet.
+__device__ __forceinline__ int len_class(int32_t len) {
+  const int tiles = len <= 0 ? 1 : (int)(((int64_t)len + kTileKeys - 1) / kTileKeys);
+  return 31 - __clz(tiles);
+}
+
+__device__ __noinline__ int seq_of_class_rank(const int32_t* lens, int B, int r,
+                                              int32_t* scratch) {
+  const int t = threadIdx.x, nt = blockDim.x, lane = t & 31, wid = t >> 5;
+  int32_t* cnt = scratch;               // [32] sequences per class
+  int32_t* wsum = scratch + 32;         // [32] per-warp totals of the scan
+  int32_t* res = scratch + 64;          // [2] class of rank r, rank within that class
+  int32_t* found = scratch + 66;        // [1] the sequence
+  if (t < 32) cnt[t] = 0;
+  __syncthreads();
+  for (int b = t; b < B; b += nt) atomicAdd(&cnt[len_class(__ldg(lens + b))], 1);
+  __syncthreads();
+  if (t == 0) {
+    int acc = 0, c = 31;
+    while (c > 0 && r >= acc + cnt[c]) acc += cnt[c--];  // r < B: stops at the class holding r
+    res[0] = c;
+    res[1] = r - acc;
+    found[0] = -1;
+  }
+  __syncthreads();
+  const int C = res[0], want = res[1];
+  const int per = (B + nt - 1) / nt;
+  const int b0 = min(B, t * per), b1 = min(B, b0 + per);
+  int mine = 0;
+  for (int b = b0; b < b1; ++b) mine += len_class(__ldg(lens + b)) == C;
+  int incl = mine;  // inclusive scan of the per-thread counts in thread order
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < wid; ++w) before += wsum[w];
+  const int start = before + incl - mine;  // class-C members in the runs before this thread's
+  if (want >= start && want < start + mine) {
+    int k = want - start;
+    for (int b = b0; b < b1; ++b)
+      if (len_class(__ldg(lens + b)) == C && k-- == 0) {
+        found[0] = b;
+        break;
+      }
+  }
+  __syncthreads();
+  return found[0];
 }
 
 // Shared-memory layout. The ring holds 16 KB slots, filled and consumed in the order K0, K1,
@@ -553,9 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t per_seq = (int64_t)a.Hkv * a.splits;
     const int64_t rem = blockIdx.x % per_seq;
     int64_t b = blockIdx.x / per_seq;
-    if (a.batch <= kRankedSeqsMax)
-      b = seq_of_rank(a.seq_lens, a.batch, (int)b,
-                      reinterpret_cast<int32_t*>(smem + C::RING_OFF));
+    int32_t* scratch = reinterpret_cast<int32_t*>(smem + C::RING_OFF);
+    b = a.batch <= kRankedSeqsMax ? seq_of_rank(a.seq_lens, a.batch, (int)b, scratch)
+                                  : seq_of_class_rank(a.seq_lens, a.batch, (int)b, scratch);
     g = (int)(rem / a.splits);
     s = (int)(rem % a.splits);
     qt = 0;

@@ -232,16 +232,17 @@ def test_gpu_decode_long_batch_sampled():
 
 @pytest.mark.gpu
 @pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
-@pytest.mark.parametrize("B", [255, 256, 257])
-def test_gpu_decode_longest_first_dispatch_edges(B):
-    """Blocks go to sequences longest first (ties by index) up to 256 sequences, in sequence
-    order beyond: both sides of that edge, with runs of equal lengths and empty sequences,
-    every output against the oracle."""
+@pytest.mark.parametrize("B,max_len,Hkv", [(255, 400, 2), (256, 400, 2), (257, 400, 2),
+                                            (700, 400, 2), (600, 6000, 1)])
+def test_gpu_decode_longest_first_dispatch_edges(B, max_len, Hkv):
+    """Blocks go to sequences longest first (ties by index) up to 256 sequences, and by length
+    class (floor(log2(KV tiles)), sequence order within a class) beyond: both sides of that
+    edge, with runs of equal lengths and empty sequences, every output against the oracle."""
     rng = np.random.default_rng(800 + B)
-    lens = rng.integers(0, 400, size=B)
+    lens = rng.integers(0, max_len, size=B)
     lens[::7] = 129          # a run of ties across the batch
     lens[3::11] = 0
-    db = decode_batch(801 + B, lens, 8, 2, 64, 16, "f16")
+    db = decode_batch(801 + B, lens, 4 * Hkv, Hkv, 64, 16, "f16")
     p, got = run_decode(db, splits=3)
     assert _binding().device_error(reset=True)[0] == 0
     empty = db.seq_lens == 0
