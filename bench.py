@@ -35,7 +35,7 @@ L2_FLUSH_BYTES = 512 << 20
 # (profiles/prefill_pair_kernel_c5_traffic.md: dram__bytes_read.sum + dram__bytes_write.sum
 # over the timed step's 16 launches / 16). It stands for the kernel whose sources hash to
 # `sources`; after any change to them the bench reports null until it is captured again.
-TRAFFIC_CAPTURE = {"workload": "c5", "sources": "2db06307b5860a2d", "bytes_per_launch": 108.58e6}
+TRAFFIC_CAPTURE = {"workload": "c5", "sources": "bfdde597adddee8b", "bytes_per_launch": 107.86e6}
 
 
 def kernel_sources_hash() -> str:
