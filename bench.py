@@ -31,11 +31,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 L2_FLUSH_BYTES = 512 << 20
 
 
-# DRAM traffic of the roofline kernel, per launch, from one ncu capture of the c5 bench step
-# (profiles/prefill_pair_kernel_c5_traffic.md: dram__bytes_read.sum + dram__bytes_write.sum
-# over the timed step's 16 launches / 16). It stands for the kernel whose sources hash to
-# `sources`; after any change to them the bench reports null until it is captured again.
-TRAFFIC_CAPTURE = {"workload": "c5", "sources": "bfdde597adddee8b", "bytes_per_launch": 107.86e6}
+# DRAM traffic of the roofline kernel, per launch: dram__bytes_read.sum + dram__bytes_write.sum
+# of one-launch ncu captures of the c5 step's prefill kernel (chunks spread over the history,
+# combined over the 16 chunks as stated in "chunks" and "how"). It stands for the kernel whose
+# sources hash to `sources`; after any change to them the bench reports null until the
+# captures are taken again.
+TRAFFIC_CAPTURE = None
 
 
 def kernel_sources_hash() -> str:
@@ -128,6 +129,29 @@ class ClockSampler:
                                    default=None)}
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first "model name" line of /proc/cpuinfo)."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def bench_config(wl, args, world: int) -> dict:
+    """The workload configuration both arms report (the same dict, so that the two lines can be
+    compared key for key)."""
+    return {"workload": wl.name, "seq_len": wl.total_keys, "chunk_rows": wl.pieces[0][1],
+            "pieces": len(wl.pieces), "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
+            "head_dim": wl.head_dim, "page_size": wl.page_size, "kv_layout": args.layout,
+            "split_policy": args.policy if args.splits is None else f"{args.splits} splits",
+            "l2": f"flushed between steps ({args.l2_flush_mb} MiB write outside the timed events)",
+            "parallelism": f"replicas x{world}"}
+
+
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
@@ -196,6 +220,9 @@ class OracleSampler:
 
 
 def reference_arm(args):
+    """The oracle as the reference arm, on the host cores of rank 0. A step is one bounded
+    stride sample of the workload's (row, head) pairs; `ms_per_step` is that sample's measured
+    wall time and `value` the query tokens of attention it covers per second."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -208,22 +235,31 @@ def reference_arm(args):
     n = sampler.calibrate(per_step)
     for k in range(warmup):
         sampler.run(max(8, n // 4), seed=50 + k)
-    rates, pairs = [], 0
+    rates, secs, pairs = [], [], 0
     for k in range(steps):
-        r, pairs, _ = sampler.run(n, seed=100 + k)
+        r, pairs, t = sampler.run(n, seed=100 + k)
         rates.append(r)
+        secs.append(t)
     cores = sampler.threads
     value = statistics.median(rates)
+    step_tokens = pairs / wl.n_q_heads
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": warmup,
-        "ms_per_step": wl.query_rows / value * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": statistics.median(secs) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "seq_len": wl.total_keys, "pieces": len(wl.pieces),
-                   "parallelism": "host cores (OpenMP)"},
+        "config": bench_config(wl, args, world),
+        "step": (f"one stride sample of {pairs} (row, head) pairs over the workload's "
+                 f"{wl.query_rows} query rows = {step_tokens:.1f} query tokens of attention; "
+                 f"ms_per_step is its measured wall time"),
+        "timed_seconds": sum(secs),
+        "workload_ms_extrapolated": wl.query_rows / value * 1e3,
+        "reference_parallelism": f"rank 0 only, {cores} host threads (OpenMP)",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "cpu_model": cpu_model(),
                          "sample": f"{pairs} (row, head) pairs per step, stride-sampled over the "
-                                   f"workload's {wl.query_rows} query rows; ~{per_step:.0f} s per step"},
+                                   f"workload's {wl.query_rows} query rows; {statistics.median(secs):.2f} s "
+                                   f"per step measured"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -475,6 +511,81 @@ def e2e_steps(inp, dw, steps, stream):
     return ms, h2d, d2h
 
 
+# The pages' long-history attention sweep (splash PR #33, "Results"): a 2048-row chunk at 32K
+# history in 512-row pieces with 4 splits (c3), and a 128-row piece at 128K history with 16
+# splits and with 1 split (c4); each also with the planner's own choice.
+SIDE_WORKLOADS = (("c3", (4, 0)), ("c4", (16, 1, 0)))
+
+
+_GENERATED = {}
+
+
+def generated(name: str):
+    """Seeded timing inputs of a workload (unused pool slots zero), made once per process."""
+    from paged_kv_long_b200.inputs import generate
+    if name not in _GENERATED:
+        _GENERATED[name] = generate(name, poison=False)
+    return _GENERATED[name]
+
+
+def workloads_measure(dev, stream, flush, peaks, reps=10):
+    """The 32K-128K configurations beside the headline: for each split setting, paged and
+    contiguous steps alternate (L2 flushed before each); per step the prefill launches are timed
+    with an event pair each on the launching stream. Reported medians: the step, the prefill
+    launches' summed time, their algorithmic TFLOP/s and fraction of the measured bf16 peak, and
+    the K/V bytes the pieces must read (every visible key's K and V row once) per second of
+    prefill-kernel time."""
+    import torch
+    from paged_kv_long_b200.inputs import WORKLOADS
+    from paged_kv_long_b200.runner import DeviceWorkload
+    res = {}
+    peak = peaks["bf16_tflops"]
+    for name, split_settings in SIDE_WORKLOADS:
+        wl = WORKLOADS[name]
+        inp = generated(name)
+        flops, kvb = wl.flops(), wl.kv_bytes()
+        t_roof = max(flops / (peak * 1e12), kvb / (peaks["hbm_gbs"] * 1e9))
+        rows = []
+        for sp in split_settings:
+            dw = DeviceWorkload(inp, dev, paged=True, splits=sp)
+            dwc = DeviceWorkload(inp, dev, paged=False, splits=sp)
+            time_steps(dw, 0, 3, flush, stream)
+            time_steps(dwc, 0, 3, flush, stream)
+            pp, cc, pk, ck = [], [], [], []
+            for _ in range(reps):
+                a_ms, a_k = time_steps(dw, 1, 0, flush, stream, record_kernels=True)
+                b_ms, b_k = time_steps(dwc, 1, 0, flush, stream, record_kernels=True)
+                pp += a_ms
+                cc += b_ms
+                pk.append(sum(a_k[0]))
+                ck.append(sum(b_k[0]))
+            torch.cuda.synchronize()
+            same = all(torch.equal(x, y) for x, y in zip(dw.outs, dwc.outs))
+            t_p, t_c = statistics.median(pp), statistics.median(cc)
+            k_p, k_c = statistics.median(pk), statistics.median(ck)
+            tf = flops / (k_p / 1e3) / 1e12
+            rows.append({
+                "splits": "planner" if sp == 0 else sp,
+                "plans": [{"policy": int(p.policy), "splits": int(p.splits), "units": int(p.units)}
+                          for p in dw.plans],
+                "paged_ms": t_p, "contiguous_ms": t_c, "paged_contiguous_ratio": t_c / t_p,
+                "query_tok_per_s": wl.query_rows / (t_p / 1e3),
+                "kernel_ms": k_p, "kernel_ms_contiguous": k_c,
+                "kernel_tflops": tf, "frac": tf / peak,
+                "kv_GB_per_s": kvb / (k_p * 1e-3) / 1e9,
+                "step_frac_of_roofline": t_roof / (t_p / 1e3),
+                "paged_contiguous_outputs_identical": bool(same)})
+            del dw, dwc
+        res[name] = {"workload": wl.name, "algorithmic_flops": flops, "algorithmic_kv_bytes": kvb,
+                     "peak_tflops": peak, "runs": rows,
+                     "how": (f"{reps} paged and {reps} contiguous steps alternating, L2 flushed "
+                             "before each; medians; kernel = the prefill launches' summed event "
+                             "time; frac = flops / kernel time / peak; kv_GB_per_s = algorithmic "
+                             "K+V bytes / kernel time")}
+        torch.cuda.empty_cache()
+    return res
+
+
 def section_arm(args):
     """One side measurement alone (for profiling it): prints its JSON object on one line."""
     import torch
@@ -544,11 +655,11 @@ def gpu_arm(args):
     t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
 
     traffic, traffic_note = None, "no capture of this kernel build"
-    if (paged and args.workload == TRAFFIC_CAPTURE["workload"] and args.policy == "makespan"
-            and args.splits is None and kernel_sources_hash() == TRAFFIC_CAPTURE["sources"]):
-        traffic = TRAFFIC_CAPTURE["bytes_per_launch"]
-        traffic_note = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, mean over the 16 "
-                        "launches of one step (cold L2 per launch under ncu), bytes per launch")
+    cap = TRAFFIC_CAPTURE
+    if (cap and paged and args.workload == cap["workload"] and args.policy == "makespan"
+            and args.splits is None and kernel_sources_hash() == cap["sources"]):
+        traffic = cap["bytes_per_launch"]
+        traffic_note = cap["how"]
 
     # ---- contiguous control at the same split counts (the ratio's denominator)
     t_contig = t_paged_pairs = last_paged = last_contig = same_bits = None
@@ -594,6 +705,11 @@ def gpu_arm(args):
     if paged and not args.no_decode:
         dec = decode_measure(wl, dev, stream, peaks)
 
+    # ---- the 32K-128K configurations (c3, c4) at the workload's and the planner's splits
+    side = None
+    if paged and not args.no_workloads and world == 1:
+        side = workloads_measure(dev, stream, flush, peaks)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e and paged:
@@ -612,8 +728,18 @@ def gpu_arm(args):
         sampler = OracleSampler(wl, inp, args.cpu_threads)
         r, pairs, t = sampler.run(sampler.calibrate(args.cpu_seconds))
         cpu = {"value": r, "unit": UNIT, "cores": sampler.threads, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"{pairs} (row, head) pairs stride-sampled over all {wl.query_rows} query "
                          f"rows of the workload, {t:.1f} s of fp64 CPU work, scaled to tok/s"}
+        if not args.no_workloads:
+            # the oracle on one thread, on the 128-row piece at 131,072 history (c4)
+            from paged_kv_long_b200.inputs import WORKLOADS
+            wl4 = WORKLOADS["c4"]
+            s1 = OracleSampler(wl4, generated("c4"), threads=1)
+            r1, p1, t1 = s1.run(s1.calibrate(3.0))
+            cpu["single_thread_c4"] = {
+                "value": r1, "unit": UNIT, "cores": 1, "gflops": r1 * wl4.flops() / wl4.query_rows / 1e9,
+                "sample": f"{p1} (row, head) pairs of c4, {t1:.1f} s on one thread"}
 
     if world > 1:
         dist.barrier()
@@ -624,13 +750,8 @@ def gpu_arm(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.name, "seq_len": wl.total_keys, "chunk_rows": wl.pieces[0][1],
-                   "pieces": len(wl.pieces), "n_q_heads": wl.n_q_heads,
-                   "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
-                   "page_size": wl.page_size, "kv_layout": args.layout,
-                   "splits": [p.splits for p in dw.plans], "split_policy": args.policy,
-                   "l2": f"flushed between steps ({args.l2_flush_mb} MiB write outside the timed events)",
-                   "parallelism": f"replicas x{world}"},
+        "config": bench_config(wl, args, world),
+        "splits_per_piece": [p.splits for p in dw.plans],
         "tflops": tflops,
         "paged_contiguous_ratio": (t_contig / t_paged_pairs) if t_contig else None,
         "paged_contiguous_ratio_last_chunk": (last_contig / last_paged) if t_contig else None,
@@ -653,6 +774,7 @@ def gpu_arm(args):
         "e2e": e2e,
         "kv_append": kv,
         "decode": dec,
+        "workloads": side,
         "staging_route": routes,
         "cpu_baseline": cpu,
         "gpu_launches": launches,
@@ -680,6 +802,8 @@ def main(argv=None):
     ap.add_argument("--no-kv-append", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-routes", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the c3/c4 side measurements (and the 1-thread oracle on c4)")
     ap.add_argument("--section", default="all", choices=["all", "decode", "kv_append", "routes"],
                     help="run one side measurement alone (1 GPU; --steps = its repetitions)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -286,7 +286,9 @@ int pa_batch_combine(const pa_plan_t* plan, const int32_t* q_lens, const int64_t
  *   device it is loaded on (PA_NOALLOC_WS_BYTES, kept until the process exits). out is
  *   written in full, as pa_prefill + pa_combine would write it.
  *   The first call on a device looks the scratch's device address up (a runtime call, made
- *   with that device current); make that first call before any stream capture.
+ *   with that device current); make that first call before any stream capture. The address
+ *   is kept for the life of the process: a device reset (cudaDeviceReset) or a teardown of
+ *   the device's primary context after that first call is not supported.
  *   Every call shares the one scratch array, which keeps the last call's contents (nothing in
  *   it needs to start at zero: each call writes every entry it reads). Calls whose work may
  *   overlap on the GPU (different streams, or several host threads without ordering) race on

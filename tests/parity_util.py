@@ -91,5 +91,24 @@ def check_sampled(inp: Inputs, outs, n=48, paged=True, what=""):
     return stats
 
 
+def all_heads(rows, Hq: int):
+    """(row, head) pairs covering every head of each given row."""
+    rows = np.asarray(rows, dtype=np.int64)
+    return np.repeat(rows, Hq), np.tile(np.arange(Hq, dtype=np.int32), len(rows))
+
+
+def oracle_rows(inp: Inputs, piece: int, rows, paged: bool = True):
+    """The oracle's outputs for every head of the given rows of one piece: (ref [n, D], pairs)."""
+    rr, hh = all_heads(rows, inp.wl.n_q_heads)
+    ref, _ = oracle.attend(oracle_problem(inp, piece, paged), rr, hh)
+    return ref, (rr, hh)
+
+
+def check_rows(got_piece: np.ndarray, ref: np.ndarray, pairs, what: str):
+    """GPU outputs of one piece at the given (row, head) pairs against the oracle's."""
+    rr, hh = pairs
+    return assert_close(got_piece[rr, hh], ref, what)
+
+
 def gen(wl, poison=True, distribution="normal"):
     return generate(wl, poison=poison, distribution=distribution)

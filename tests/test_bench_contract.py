@@ -30,6 +30,16 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert "workload" in d["config"]
+    # the same config dict as the GPU arm on the same arguments
+    from paged_kv_long_b200.inputs import WORKLOADS
+    args = bench.main.__globals__["argparse"].Namespace(layout="paged", policy="makespan",
+                                                          splits=None,
+                                                          l2_flush_mb=bench.L2_FLUSH_BYTES >> 20)
+    assert d["config"] == bench.bench_config(WORKLOADS["c1"], args, 1)
+    # ms_per_step is the measured wall time of one sampled step, so the steps add up to the
+    # timed seconds the line reports
+    assert abs(d["ms_per_step"] * d["steps"] / 1e3 - d["timed_seconds"]) <= 0.5 * d["timed_seconds"]
+    assert d["cpu_baseline"]["cpu_model"]
 
 
 def test_warmup_below_three_is_refused():
@@ -40,4 +50,5 @@ def test_warmup_below_three_is_refused():
 def test_traffic_capture_is_keyed_to_the_kernel_sources():
     h = bench.kernel_sources_hash()
     assert len(h) == 16 and int(h, 16) >= 0
-    assert set(bench.TRAFFIC_CAPTURE) == {"workload", "sources", "bytes_per_launch"}
+    cap = bench.TRAFFIC_CAPTURE
+    assert cap is None or set(cap) == {"workload", "sources", "bytes_per_launch", "how"}

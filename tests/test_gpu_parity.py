@@ -217,30 +217,51 @@ def test_argument_errors():
 
 
 # ------------------------------------------------------------------ the five workloads, full size
-def test_c3_full_size_sampled():
+# Dense at full size: c4's 3,072 outputs all, under 16 splits (the workload's), 1 split and the
+# planner's items; the last piece of c3 and the last chunk of c5 on every 8th row, all heads;
+# the other pieces of c3 on seeded samples and the other chunks of c5 on every 64th row, all
+# heads. Relative RMS is taken over each compared set.
+def test_c3_full_size_dense_last_piece():
     inp = U.gen("c3")
     _, outs = U.run_gpu(inp)                 # 4 splits per piece, as the workload states
-    U.check_sampled(inp, outs, what="c3 S=4")
-    _, outp = U.run_gpu(inp, splits=0)      # the planner's split count
-    U.check_sampled(inp, outp, n=16, what="c3 planned")
+    _, outp = U.run_gpu(inp, splits=0)      # the planner's split count (balanced items)
+    last = len(inp.wl.pieces) - 1
+    ref, pairs = U.oracle_rows(inp, last, np.arange(0, inp.wl.pieces[last][1], 8))
+    U.check_rows(outs[last], ref, pairs, "c3 S=4 last piece, every 8th row")
+    U.check_rows(outp[last], ref, pairs, "c3 planned last piece, every 8th row")
+    for i in range(last):
+        rows, heads = U.sample_pairs(inp.wl.pieces[i][1], inp.wl.n_q_heads, 48, 7919 + i, 6)
+        ref_i, _ = U.oracle.attend(U.oracle_problem(inp, i), rows, heads)
+        U.assert_close(outs[i][rows, heads], ref_i, f"c3 S=4 piece {i} sampled")
+        U.assert_close(outp[i][rows, heads], ref_i, f"c3 planned piece {i} sampled")
     _, outc = U.run_gpu(inp, paged=False)
     for a, b in zip(outs, outc):
         assert np.array_equal(a, b)
 
 
-def test_c4_full_size_sampled():
+def test_c4_full_size_every_output():
     inp = U.gen("c4")
+    ref, pairs = U.oracle_rows(inp, 0, np.arange(inp.wl.pieces[0][1]))   # 128 rows x 24 heads
     _, o16 = U.run_gpu(inp)                  # 16 splits + combine
-    U.check_sampled(inp, o16, n=64, what="c4 S=16")
+    U.check_rows(o16[0], ref, pairs, "c4 S=16, every output")
     _, o1 = U.run_gpu(inp, splits=1)
-    U.check_sampled(inp, o1, n=32, what="c4 S=1")
+    U.check_rows(o1[0], ref, pairs, "c4 S=1, every output")
+    dw, op = U.run_gpu(inp, splits=0)        # the planner's items
+    assert dw.plans[0].policy == binding.PA_POLICY_BALANCED
+    U.check_rows(op[0], ref, pairs, "c4 planned, every output")
     assert np.abs(o1[0].astype(np.float64) - o16[0]).max() <= 2.0 ** -10
+    _, oc = U.run_gpu(inp, paged=False)
+    assert np.array_equal(o16[0], oc[0])
 
 
-def test_c5_full_size_sampled_paged_equals_contiguous():
+def test_c5_full_size_dense_paged_equals_contiguous():
     inp = U.gen("c5")
     _, outs = U.run_gpu(inp)                 # planner's split count per chunk
-    U.check_sampled(inp, outs, n=24, what="c5 paged")
+    n = len(inp.wl.pieces)
+    for i, (h, r) in enumerate(inp.wl.pieces):
+        step = 8 if i == n - 1 else 64
+        ref, pairs = U.oracle_rows(inp, i, np.arange(i % step, r, step))
+        U.check_rows(outs[i], ref, pairs, f"c5 chunk {i} (H={h}), every {step}th row")
     _, outc = U.run_gpu(inp, paged=False)
     for a, b in zip(outs, outc):
         assert np.array_equal(a, b)
