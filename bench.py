@@ -354,7 +354,25 @@ def kv_append_measure(inp, dev, stream, peaks, reps=20):
             torch.cuda.synchronize()
             return e0.elapsed_time(e1) / reps
 
-        t_all = timed(lambda: binding.kv_append(kn, vn, kp, vp, tab, h0, stream))
+        t_pair = timed(lambda: binding.kv_append(kn, vn, kp, vp, tab, h0, stream))
+
+        def graphed(fn, n):
+            """n calls captured in one CUDA graph, replayed between one event pair: the kernel's
+            time per call with the launch gaps of a graph, not the event-to-kernel latency."""
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    fn(torch.cuda.current_stream())
+            for _ in range(2):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n
+
+        t_all = graphed(lambda st: binding.kv_append(kn, vn, kp, vp, tab, h0, st), reps)
 
         def chunks():
             for h, r in wl.pieces:
@@ -364,8 +382,11 @@ def kv_append_measure(inp, dev, stream, peaks, reps=20):
     nbytes = 2 * rows * wl.n_kv_heads * wl.head_dim * 2 * 2   # K and V, read once, written once
     gbs = nbytes / (t_all * 1e-3) / 1e9
     return {"workload": f"{rows} rows of K and V (all the workload's positions) in one call",
-            "timing": "an event pair around each call, median of the calls",
-            "ms": t_all, "GB_per_s": gbs, "peak_GB_per_s": peaks["hbm_gbs"],
+            "timing": (f"{reps} calls replayed as one CUDA graph between an event pair, per call; "
+                       "ms_event_pair: an event pair around each eager call, median (it adds "
+                       "the event-to-kernel latency)"),
+            "ms": t_all, "ms_event_pair": t_pair, "GB_per_s": gbs,
+            "peak_GB_per_s": peaks["hbm_gbs"],
             "frac": gbs / peaks["hbm_gbs"], "bytes": nbytes,
             "us_per_chunk_call_host_bound": t_chunks * 1e3 / len(wl.pieces),
             "chunk_calls": len(wl.pieces)}
@@ -586,6 +607,37 @@ def workloads_measure(dev, stream, flush, peaks, reps=10):
     return res
 
 
+def pieces_run(wl, dev, stream, args):
+    """Some pieces of a workload alone (for one-launch profiler captures): every listed piece's
+    prefill + combine `--steps` times in turn (L2 flushed before each), in the chosen layout and
+    split setting. Launch order: piece p0's prefill, its merge (if split), piece p1's ...; the
+    first (steps - 1) rounds are warm-up for a capture of the last round."""
+    import torch
+    from paged_kv_long_b200.runner import DeviceWorkload
+    inp = generated(args.workload)
+    dw = DeviceWorkload(inp, dev, paged=args.layout == "paged", splits=args.splits,
+                        policy=args.policy)
+    idx = [int(x) for x in args.pieces.split(",")] if args.pieces else list(range(len(wl.pieces)))
+    flush = torch.empty(max(args.l2_flush_mb, 1) * (1 << 20) // 4, dtype=torch.float32,
+                        device=dev)
+    ms = {i: [] for i in idx}
+    for _ in range(args.steps):
+        for i in idx:
+            with torch.cuda.stream(stream):
+                flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dw.run_piece(i, stream)
+            e1.record(stream)
+            ms[i].append((e0, e1))
+    torch.cuda.synchronize()
+    return {"workload": wl.name, "layout": args.layout,
+            "pieces": {str(i): {"hist_len": wl.pieces[i][0], "rows": wl.pieces[i][1],
+                                "splits": int(dw.plans[i].splits), "policy": int(dw.plans[i].policy),
+                                "units": int(dw.plans[i].units),
+                                "ms": [a.elapsed_time(b) for a, b in ms[i]]} for i in idx}}
+
+
 def section_arm(args):
     """One side measurement alone (for profiling it): prints its JSON object on one line."""
     import torch
@@ -594,7 +646,9 @@ def section_arm(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.Stream(dev)
     peaks = load_peaks()
-    if args.section == "decode":
+    if args.section == "piece":
+        res = pieces_run(wl, dev, stream, args)
+    elif args.section == "decode":
         res = decode_measure(wl, dev, stream, peaks, reps=args.steps)
     else:
         inp = generate(wl, poison=False)
@@ -804,8 +858,11 @@ def main(argv=None):
     ap.add_argument("--no-routes", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the c3/c4 side measurements (and the 1-thread oracle on c4)")
-    ap.add_argument("--section", default="all", choices=["all", "decode", "kv_append", "routes"],
-                    help="run one side measurement alone (1 GPU; --steps = its repetitions)")
+    ap.add_argument("--section", default="all",
+                    choices=["all", "decode", "kv_append", "routes", "piece"],
+                    help="run one side measurement alone (1 GPU; --steps = its repetitions); "
+                         "'piece' runs the pieces listed by --pieces")
+    ap.add_argument("--pieces", default="", help="piece indices for --section piece, e.g. 0,7,15")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--cpu-threads", type=int, default=0,

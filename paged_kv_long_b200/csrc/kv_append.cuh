@@ -5,25 +5,47 @@
 //
 // Position p = H + i of chunk row i lives in page page_table[p / PS], slot p % PS. A pool slot
 // [page][slot] holds all KV heads of one position contiguously (Hkv * D 16-bit values), so a
-// row is one contiguous copy. One warp copies one row of K or of V in 16-byte pieces; the work
-// is HBM-bound (each byte read once and written once).
+// row is one contiguous copy. One warp copies one position: its K row and its V row (the same
+// page slot, one page-table read), in 16-byte pieces, with every load of a batch of up to four
+// pieces per lane and tensor issued before its stores (up to eight loads in flight per lane).
+// The work is HBM-bound (each byte read once and written once).
 
 __global__ void __launch_bounds__(256) kv_append_kernel(
     const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_pool,
     uint4* __restrict__ v_pool, const int32_t* __restrict__ page_table, int64_t num_pages,
     int64_t hist_len, int64_t rows, int page_size, int row_vecs) {
-  const int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  if (w >= 2 * rows) return;
+  const int64_t i = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (i >= rows) return;
   const int lane = threadIdx.x & 31;
-  const int64_t i = w >> 1;
-  const bool is_v = (w & 1) != 0;
   const int64_t pos = hist_len + i;
   const int32_t e = __ldg(page_table + pos / page_size);
   if (e < 0 || e >= num_pages) {  // skipped, reported through the device error word
     if (lane == 0) atomicOr(&g_pa_error_flags, kFlagPage);
     return;
   }
-  const uint4* src = (is_v ? v_new : k_new) + i * row_vecs;
-  uint4* dst = (is_v ? v_pool : k_pool) + ((int64_t)e * page_size + pos % page_size) * row_vecs;
-  for (int c = lane; c < row_vecs; c += 32) dst[c] = __ldg(src + c);
+  const uint4* ks = k_new + i * row_vecs;
+  const uint4* vs = v_new + i * row_vecs;
+  const int64_t slot = ((int64_t)e * page_size + pos % page_size) * row_vecs;
+  uint4* kd = k_pool + slot;
+  uint4* vd = v_pool + slot;
+  constexpr int kBatch = 4;
+  for (int c0 = 0; c0 < row_vecs; c0 += 32 * kBatch) {
+    uint4 kv[kBatch], vv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + lane + 32 * u;
+      if (c < row_vecs) {
+        kv[u] = __ldg(ks + c);
+        vv[u] = __ldg(vs + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + lane + 32 * u;
+      if (c < row_vecs) {
+        kd[c] = kv[u];
+        vd[c] = vv[u];
+      }
+    }
+  }
 }

@@ -349,6 +349,41 @@ struct SoftmaxCtx {
   uint64_t tmo;
 };
 
+// Epilogue of one softmax thread (packed row r of its CTA's Q tile, tensor-memory lane
+// t_lane): O / l from tensor memory to the output row, or to the workspace row of a partial
+// together with its base-2 log-sum-exp. The row goes through shared memory (x.stage_off, idle
+// once the last P V is done; rows 16 bytes apart from a multiple of 128 so that a warp's
+// stores spread over the banks) and leaves as one contiguous bulk copy.
+template <int D>
+__device__ __forceinline__ void write_row(const PrefillArgs& a, const SoftmaxCtx& x, int r,
+                                          bool valid, int64_t tok, int head, float m_run,
+                                          float l_run, uint32_t t_lane) {
+  const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+  int64_t ws_row = -1;  // workspace row of a partial; -1: the final output
+  if (x.slot >= 0)
+    ws_row = (int64_t)x.slot * a.rows_per_block + x.row0 + r;
+  else if (x.slot == kSlotUniform && a.splits > 1)
+    ws_row = (int64_t)x.s * a.ws_split_rows + tok * a.Hq + head;
+  float* dst = ws_row < 0 ? a.out + (tok * a.Hq + head) * (int64_t)D : a.ws_o + ws_row * D;
+  const uint32_t srow = x.sb + x.stage_off + (uint32_t)r * (uint32_t)(D * 4 + 16);
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    float o[32];
+    tmem_ld32(t_lane + kOCol + 32u * c, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      st_shared_v4(srow + 128u * c + 16u * i, __float_as_uint(o[4 * i] * inv_l),
+                   __float_as_uint(o[4 * i + 1] * inv_l), __float_as_uint(o[4 * i + 2] * inv_l),
+                   __float_as_uint(o[4 * i + 3] * inv_l));
+  }
+  fence_proxy_async_smem();
+  if (valid) bulk_store(dst, srow, D * 4);
+  bulk_commit();
+  bulk_wait_read_all();
+  if (valid && ws_row >= 0) a.ws_lse[ws_row] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+}
+
 template <int D, bool PAGED, bool BF16, class VTail>
 __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const SoftmaxCtx& x,
                                              VTail&& v_tail) {
@@ -356,7 +391,7 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sb = x.sb, tmem = x.tmem;
   const int64_t qt = x.qt, kt0 = x.kt0;
-  const int g = x.g, s = x.s, n = x.n;
+  const int g = x.g, n = x.n;
   volatile int* abort_flag = x.abort_flag;
   const uint64_t tmo = x.tmo;
   auto arrive = [&](uint32_t addr) {
@@ -520,33 +555,7 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
                      g_pa_units[kUnitWords * blockIdx.x + 6] = clock64();)
     if (ok) {
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      int64_t ws_row = -1;  // workspace row of a partial; -1: the final output
-      if (x.slot >= 0)
-        ws_row = (int64_t)x.slot * a.rows_per_block + x.row0 + r;
-      else if (x.slot == kSlotUniform && a.splits > 1)
-        ws_row = (int64_t)s * a.ws_split_rows + tok * a.Hq + head;
-      float* dst = ws_row < 0 ? a.out + (tok * a.Hq + head) * (int64_t)D : a.ws_o + ws_row * D;
-      // The row goes through shared memory (the K/V ring, idle now; rows 16 bytes apart from
-      // a multiple of 128 so a warp's stores spread over the banks) and leaves as one
-      // contiguous bulk copy per row.
-      const uint32_t srow = sb + x.stage_off + (uint32_t)r * (uint32_t)(D * 4 + 16);
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(t_lane + kOCol + 32u * c, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_shared_v4(srow + 128u * c + 16u * i, __float_as_uint(o[4 * i] * inv_l),
-                       __float_as_uint(o[4 * i + 1] * inv_l), __float_as_uint(o[4 * i + 2] * inv_l),
-                       __float_as_uint(o[4 * i + 3] * inv_l));
-      }
-      fence_proxy_async_smem();
-      if (valid) bulk_store(dst, srow, D * 4);
-      bulk_commit();
-      bulk_wait_read_all();
-      if (valid && ws_row >= 0) a.ws_lse[ws_row] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+      write_row<D>(a, x, r, valid, tok, head, m_run, l_run, t_lane);
     }
     PA_TRACE_ONLY(tr[2] += clock64() - te;
                   if (lane == 0) {
@@ -1177,7 +1186,7 @@ cudaError_t launch_pair(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
   cfg.dynamicSmemBytes = PairCfg::LAUNCH_SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1620,7 +1629,7 @@ extern "C" int pa_kv_append(int n_kv_heads, int head_dim, int page_size, int dty
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
     return PA_ERR_INVALID_ARG;
   const int row_vecs = n_kv_heads * head_dim * 2 / 16;
-  const int64_t warps = 2 * (int64_t)chunk_rows;
+  const int64_t warps = chunk_rows;  // one per position (its K and V rows)
   const int64_t blocks = (warps + 7) / 8;
   if (blocks >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   kv_append_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(

@@ -1,21 +1,46 @@
 // prefill_pair.cuh — the head-dim-256 prefill kernel on CTA pairs (a cluster of two CTAs whose
 // tensor cores work as one, tcgen05 cta_group::2). Included by pa_kernels.cu.
 //
-// A unit is (KV head, pair of packed Q tiles, history split). CTA rank r of the pair holds
-// Q tile 2t+r (its own 128 rows): its Q in shared memory, its S/P and O in its own tensor
-// memory, and its softmax warps. Rank 0 issues every MMA of the pair with M = 256:
-//   S = Q K^T:  A = the two Q tiles, B = K split by keys (rank r holds keys 64r..64r+63 of
-//               each 128-key tile, all 256 of D);
-//   O += P V:   A = the two P tiles (each in its own tensor memory), B = V split by D (rank r
-//               holds dims 128r..128r+127 of all 128 keys).
-// Each CTA therefore loads half of every K/V tile: half the L2 traffic per FLOP of the
-// single-CTA kernel, and twice the time its shared-memory ring covers. Each CTA's copies fill
-// its own shared memory, and both halves of a slot complete on rank 0's barrier (the pair form
-// of the tensor copy), so rank 0 sees a slot as one unit. Rank 1 tells rank 0 when its Q and P
-// are ready (remote mbarrier arrivals); rank 0's MMA completions reach both CTAs (multicast
-// commits). One exception: the V rows of the sequence's last, partly filled tile complete on
-// the issuing CTA's own barrier, because its softmax warps zero the rows past the end before
-// the PV product reads them.
+// A unit is (KV head, pair of packed Q tiles, history split) or a balanced work item. CTA rank
+// r of the pair holds Q tile 2t+r (its own 128 rows): its Q in shared memory, its S, P and O
+// in its own tensor memory, and its softmax warps. Rank 0 issues every MMA of the pair with
+// M = 256:
+//   S = Q K^T:  A = the two Q tiles (shared memory), B = K split by keys (rank r holds keys
+//               64r..64r+63 of each 128-key tile, all 256 of D);
+//   O += P V:   A = the two P tiles (tensor memory), B = V split by D (rank r holds dims
+//               128r..128r+127 of all 128 keys).
+// Each CTA therefore loads half of every K/V tile. Each CTA's copies fill its own shared
+// memory, and both halves of a slot complete on rank 0's barrier (the pair form of the tensor
+// copy), so rank 0 sees a slot as one unit; rank 0's MMA completions reach both CTAs
+// (multicast commits).
+//
+// The tile loop. Tensor memory (512 columns) holds O (256), one S buffer (128) and two P
+// buffers (64 columns of 16-bit pairs each). The softmax warps read S(j) into registers and
+// release the buffer at once (s_free), so that QK(j+1) runs while the softmax of tile j does;
+// P(j) goes to P buffer j % 2, which the softmax writes once PV(j-2) (its last reader) is
+// done. Two threads of rank 0 issue the MMAs: one every QK, the other every PV.
+// tcgen05.mma holds its issuing thread until the tensor pipe takes the instruction, so a
+// single issuer leaves the pipe idle through every wait and commit between its MMA groups
+// (measured: ~900 of ~3,100 cycles per tile); with two, one stream feeds the pipe while the
+// other waits, and QK and PV (different accumulators) interleave. Copies land in a ring of
+// ten 16 KB slots in the order K0, K1, then per tile j, K(j+2) and V(j); each issuer finds its
+// slots from these positions.
+//
+// Rank 1's softmax warps announce the end of their S reads and their P to rank 0 with
+// CTA-scope remote arrivals (tensor-memory accesses, ordered by tcgen05.wait and the
+// before-thread-sync fence). Where they also wrote their CTA's shared memory (a Q tile loaded
+// by the threads; V rows zeroed in the last tile) each thread makes the writes visible to the
+// async proxy and releases them at cluster scope with a fence restricted to its own CTA's
+// shared memory before a relaxed cluster-scope arrival (a full cluster-scope release measured
+// ~1,400 cycles). The V rows of the sequence's last, partly filled tile complete on the
+// issuing CTA's own barrier, because its softmax warps zero the rows past the end before the
+// PV product reads them.
+
+constexpr int kPairThreads = 256;    // warps: 0-3 softmax, 4 QK issuer, 5-6 copies, 7 PV issuer
+constexpr int kPairPvWarp = 7;
+constexpr int kPairIssuers = 2;      // copy-issuing warps
+constexpr uint32_t kPairSCol = 256;  // S: one buffer of 128 columns
+constexpr uint32_t kPairPCol = 384;  // P: buffers of 64 columns (16-bit pairs) at 384 and 448
 
 struct PairCfg {
   static constexpr int NP = 4;        // 64-wide panels of a 256-wide row
@@ -23,15 +48,18 @@ struct PairCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NP * kPanel;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * kPanel;
-  // full[10] (rank 0: both halves landed), empty[10], q_full, s_full[2], p_full[2],
-  // pv_done[2], mma_done, teardown
+  // full[10] (rank 0: both halves landed), empty[10], q_full, s_full, s_free, p_full[2],
+  // pv_done[2], mma_done (both issuers' last commits), teardown
   static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_QFULL = 2 * NSLOT,
-                       B_SFULL = 2 * NSLOT + 1, B_PFULL = 2 * NSLOT + 3, B_PVDONE = 2 * NSLOT + 5,
-                       B_MMADONE = 2 * NSLOT + 7, B_TEAR = 2 * NSLOT + 8, N_BARS = 2 * NSLOT + 9;
+                       B_SFULL = 2 * NSLOT + 1, B_SFREE = 2 * NSLOT + 2, B_PFULL = 2 * NSLOT + 3,
+                       B_PVDONE = 2 * NSLOT + 5, B_MMADONE = 2 * NSLOT + 7,
+                       B_TEAR = 2 * NSLOT + 8, N_BARS = 2 * NSLOT + 9;
   static constexpr int MISC_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int SMEM = MISC_OFF + 16;
   static constexpr int LAUNCH_SMEM = SMEM + 1024;
   static_assert(LAUNCH_SMEM <= 232448, "exceeds 227 KB of shared memory per CTA");
+  // the epilogue stages 128 rows of 1 KB (+16 B) over the ring, idle by then
+  static_assert(NSLOT * kPanel >= kTileRows * (256 * 4 + 16), "staging needs the ring");
 };
 
 // Byte offset inside a V half tile (2 slots: keys 0-63, then 64-127) of key row k, local panel
@@ -42,8 +70,201 @@ __device__ __forceinline__ uint32_t v_offset_pair(uint32_t k, uint32_t pl, int v
          ((kk & ((1u << v_shift) - 1u)) << 7);
 }
 
+// Positions of the half tiles in the ring's fill order K0, K1, then per tile j: K(j+2) (while
+// j + 2 < n), V(j). K tile m and V tile j of a unit of n tiles:
+__device__ __forceinline__ uint32_t pair_k_item(int m) { return m <= 1 ? (uint32_t)m : 2u * m - 2u; }
+__device__ __forceinline__ uint32_t pair_v_item(int j, int n) {
+  return j <= n - 3 ? 2u * j + 3u : (j == n - 2 ? 2u * n - 2u : 2u * n - 1u);
+}
+
+// Barriers of the pair's softmax warps besides those of SoftmaxCtx.
+struct PairSync {
+  uint32_t arrive_sfree;  // s_free of rank 0 (remote on rank 1)
+  uint32_t arrive_p;      // p_full[0] of rank 0 (remote on rank 1); +8: buffer 1
+};
+
+// Softmax + epilogue warps of the pair kernel (warps 0-3, one thread per packed Q row of this
+// CTA's tile = tensor-memory lane).
+template <bool PAGED, bool BF16, class VTail>
+__device__ __forceinline__ void softmax_pair_role(const PrefillArgs& a, const SoftmaxCtx& x,
+                                                  const PairSync& y, VTail&& v_tail) {
+  constexpr int D = 256;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tmem = x.tmem;
+  const int64_t qt = x.qt, kt0 = x.kt0;
+  const int g = x.g, n = x.n;
+  volatile int* abort_flag = x.abort_flag;
+  const uint64_t tmo = x.tmo;
+  const int r = threadIdx.x;  // packed Q row = tensor-memory lane
+  const int64_t grow = qt * kTileRows + r;
+  const int64_t tok = grow / a.G;
+  const bool valid = tok < a.R;
+  const int head = g * a.G + (int)(grow % a.G);
+  const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+  if (!a.q_tma) {
+    // Q tile -> shared memory as K-major rows of 64-element panels, 128-byte swizzle (when the
+    // tensor copy cannot: it loads whole tokens, so it needs G to divide 128).
+    const uint4* src =
+        reinterpret_cast<const uint4*>(a.q + (valid ? (tok * a.Hq + head) * (int64_t)D : 0));
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = valid ? __ldg(src + p * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+        st_shared_v4(x.sb + x.q_off + p * kPanel + r * 128 + ((c ^ (r & 7)) << 4), v.x, v.y,
+                     v.z, v.w);
+      }
+    }
+    fence_proxy_async_smem();
+    if (x.remote_arrive) fence_release_smem_cluster();
+    __syncwarp();
+    if (lane == 0) {
+      if (x.remote_arrive)
+        mbar_arrive_remote_relaxed(x.arrive_qfull);
+      else
+        mbar_arrive(x.arrive_qfull);
+    }
+  }
+
+  const int64_t limit = valid ? a.hist_len + tok : -1;  // last key this row may see
+  const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+  float m_run = -INFINITY;  // running max of scale*log2(e)*score
+  float l_run = 0.f;        // running sum of the probabilities (fp32)
+  bool ok = true;
+  // PV of tile i completes phase (i / 2) % 2 of pv_done[i % 2]. The softmax waits for PV(i)
+  // only at tiles i + 1 (a rescale of O) and i + 2 (P's buffer); the next completion on that
+  // barrier, PV(i + 2), needs P(i + 2), stored after those waits, so no parity wait skips a
+  // phase.
+  auto wait_pv = [&](int i) -> bool {
+    return warp_wait(x.bar_pvdone + 8u * (uint32_t)(i & 1), (uint32_t)(i >> 1) & 1u, abort_flag,
+                     tmo);
+  };
+  for (int j = 0; j < n; ++j) {
+    const int64_t key0 = (kt0 + j) * kTileKeys;
+    if (!warp_wait(x.bar_sfull, (uint32_t)j & 1u, abort_flag, tmo)) {
+      ok = false;
+      break;
+    }
+    PA_UNIT_ONLY(if (j == 0 && threadIdx.x == 0 && blockIdx.x < 8192)
+                     g_pa_units[kUnitWords * blockIdx.x + 5] = clock64();)
+    tc_fence_after();
+    float sv[kTileKeys];
+#pragma unroll
+    for (int c = 0; c < kTileKeys / 32; ++c)
+      tmem_ld32(t_lane + kPairSCol + 32u * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
+    tmem_wait_ld();
+    // S(j) is in registers: the buffer may take S(j+1)
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      if (x.remote_arrive)
+        mbar_arrive_remote_tc(y.arrive_sfree);
+      else
+        mbar_arrive(y.arrive_sfree);
+    }
+
+    // causal mask by select (masked scores become -inf, whatever bits they held)
+    const int64_t rel64 = limit - key0;
+    if (rel64 < kTileKeys - 1) {
+      const int rel = rel64 < -1 ? -1 : (int)rel64;
+#pragma unroll
+      for (int c = 0; c < kTileKeys; ++c)
+        if (c > rel) sv[c] = -INFINITY;
+    }
+    // row max: eight independent chains, then a tree
+    float mx8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+#pragma unroll
+    for (int c = 8; c < kTileKeys; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+    const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+    const float m_new = fmaxf(m_run, mx * a.scale_log2);
+    const bool need = m_new > m_run + kRescaleLog2;
+    // The probabilities use the new reference whenever it moves; O (and l) are brought to it
+    // below, once the PV that last wrote O has completed.
+    const float f_resc = (need && m_run != -INFINITY) ? ex2(m_run - m_new) : 1.0f;
+    if (need) m_run = m_new;
+    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+    const float2 nm2 = make_float2(-m_use, -m_use);
+    float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                    make_float2(0.f, 0.f)};
+    uint32_t pk[kTileKeys / 2];
+#pragma unroll
+    for (int c = 0; c < kTileKeys; c += 2) {
+      const float2 t = ffma2(make_float2(sv[c], sv[c + 1]), sc2, nm2);
+      const float2 pr = make_float2(ex2(t.x), ex2(t.y));
+      ls[(c >> 1) & 3] = fadd2(ls[(c >> 1) & 3], pr);
+      pk[c >> 1] = pack2<BF16>(pr.x, pr.y);
+    }
+    const float l_tile = (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y) + (ls[2].x + ls[2].y) +
+                         (ls[3].x + ls[3].y);
+    if (j >= 1 && __any_sync(0xffffffffu, f_resc != 1.0f)) {
+      // O must not change under a running MMA: wait for PV(j-1), the last to write it
+      if (!wait_pv(j - 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(t_lane + kOCol + 32u * c, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= f_resc;
+        tmem_st32(t_lane + kOCol + 32u * c, o);
+      }
+      tmem_wait_st();
+    }
+    l_run = l_run * f_resc + l_tile;
+    // P's buffer j % 2 was last read by PV(j-2)
+    if (j >= 2 && !wait_pv(j - 2)) {
+      ok = false;
+      break;
+    }
+
+    // The sequence's last tile, partly past its end (paged pools): this CTA's half of the V
+    // rows past the end is zeroed in shared memory before PV reads it.
+    const bool tail = PAGED && key0 + kTileKeys > a.total_keys;
+    if (tail && !v_tail(j, key0 + r >= a.total_keys ? r : -1)) {
+      ok = false;
+      break;
+    }
+    // P(j) (rounded to the input type) into P buffer j % 2: one row per lane, 16-bit pairs
+    const uint32_t p_col = kPairPCol + 64u * (uint32_t)(j & 1);
+    tmem_st32u(t_lane + p_col, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+    tmem_st32u(t_lane + p_col + 32u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+    tmem_wait_st();
+    tc_fence_before();
+    if (tail) {
+      fence_proxy_async_smem();
+      if (x.remote_arrive) fence_release_smem_cluster();
+    }
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t pb = y.arrive_p + 8u * (uint32_t)(j & 1);
+      if (!x.remote_arrive)
+        mbar_arrive(pb);
+      else if (tail)
+        mbar_arrive_remote_relaxed(pb);
+      else
+        mbar_arrive_remote_tc(pb);
+    }
+  }
+
+  if (ok && n >= 2) ok = wait_pv(n - 2);
+  if (ok) ok = wait_pv(n - 1);
+  PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
+                   g_pa_units[kUnitWords * blockIdx.x + 6] = clock64();)
+  if (ok) {
+    tc_fence_after();
+    write_row<D>(a, x, r, valid, tok, head, m_run, l_run, t_lane);
+  }
+}
+
 template <bool PAGED, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_q, const PrefillArgs a_in,
@@ -95,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The copy warps read the page-table entries of the first two KV tiles before the set-up
   // below, so the loads overlap it and the first copies go out right after it.
   int32_t pre_row0 = a.oob_row, pre_row1 = a.oob_row;
-  if (warp > kMmaWarp) {
+  if (warp > kMmaWarp && warp < kPairPvWarp) {
     const bool report = warp == kMmaWarp + 1;
     pre_row0 = tile_page_row<PAGED>(a, kt0, n, 0, lane, report);
     pre_row1 = tile_page_row<PAGED>(a, kt0, n, 1, lane, report);
@@ -120,13 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Q by tensor copy: one arrival (rank 0's, with both CTAs' bytes); else 4 softmax warps
     // here + 4 of rank 1
     mbar_init(bar(C::B_QFULL), a.q_tma ? 1 : 8);
-    mbar_init(bar(C::B_SFULL + 0), 1);
-    mbar_init(bar(C::B_SFULL + 1), 1);
-    mbar_init(bar(C::B_PFULL + 0), 8);
+    mbar_init(bar(C::B_SFULL), 1);
+    mbar_init(bar(C::B_SFREE), 8);      // 4 softmax warps here + 4 of rank 1
+    mbar_init(bar(C::B_PFULL + 0), 8);  // 4 softmax warps here + 4 of rank 1
     mbar_init(bar(C::B_PFULL + 1), 8);
     mbar_init(bar(C::B_PVDONE + 0), 1);
     mbar_init(bar(C::B_PVDONE + 1), 1);
-    mbar_init(bar(C::B_MMADONE), 1);
+    mbar_init(bar(C::B_MMADONE), 2);
     mbar_init(bar(C::B_TEAR), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -149,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                    g_pa_units[kUnitWords * blockIdx.x + 4] = clock64();)
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
-  PA_TRACE_ONLY(unsigned tln = 0;)
 
   // Cluster-scope bounded wait (for barriers the other CTA arrives on).
   auto wait_cluster = [&](uint32_t b, uint32_t parity) -> bool {
@@ -177,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.bar_pvdone = bar(C::B_PVDONE);
     sc.remote_arrive = rank != 0;
     sc.arrive_qfull = rank == 0 ? bar(C::B_QFULL) : leader_bar(C::B_QFULL);
-    sc.arrive_pfull = rank == 0 ? bar(C::B_PFULL) : leader_bar(C::B_PFULL);
+    sc.arrive_pfull = 0;
     sc.tmem = tmem;
     sc.qt = qt;
     sc.g = g;
@@ -187,15 +407,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     sc.slot = slot;
     sc.row0 = (int)rank * kTileRows;
     sc.stage_off = C::RING_OFF;
-    static_assert(NSLOT * kPanel >= kTileRows * (D * 4 + 16), "staging needs the ring");
     sc.abort_flag = abort_flag;
     sc.tmo = tmo;
+    PairSync ps;
+    ps.arrive_sfree = rank == 0 ? bar(C::B_SFREE) : leader_bar(C::B_SFREE);
+    ps.arrive_p = rank == 0 ? bar(C::B_PFULL) : leader_bar(C::B_PFULL);
     // Keys past the sequence in its last page hold arbitrary bits; P is 0 there but 0 * NaN
     // is NaN inside the MMA, so this CTA's half of those V rows is zeroed before PV.
     // Those fills complete on this CTA's own barrier: on rank 1 that barrier sees no other
     // phase, so its parity is 0.
     auto v_tail = [&](int j, int r) -> bool {
-      const uint32_t seq0 = v_item(j, n) * 2;
+      const uint32_t seq0 = pair_v_item(j, n) * 2;
       bool okv = true;
       for (int k = 0; k < 2 && okv; ++k)
         okv = warp_wait(bar(C::B_FULL + (seq0 + k) % NSLOT),
@@ -207,14 +429,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) st_shared_v4(ra + c * 16, 0u, 0u, 0u, 0u);
       }
-      fence_proxy_async_smem();
       return true;
     };
-    softmax_role<D, PAGED, BF16>(a, sc, v_tail);
-  } else if (warp > kMmaWarp) {
-    // ============================================================ TMA issuers (three warps)
-    // Fill q (2 per K or V half tile, in the order K0, K1, V0, K2, V1, ...) is issued by warp
-    // q % kIssuers; lanes issue one box each.
+    softmax_pair_role<PAGED, BF16>(a, sc, ps, v_tail);
+  } else if (warp > kMmaWarp && warp < kPairPvWarp) {
+    // ============================================================ TMA issuers (two warps)
+    // Fill q (2 per K or V half tile, in the order of pair_k_item / pair_v_item) is issued by
+    // warp q % kPairIssuers; lanes issue one box each.
     const int w = warp - kMmaWarp - 1;
     const int ppt = a.pages_per_tile;
     const int prow = a.page_rows;
@@ -250,7 +471,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the tail fills.
     auto acquire = [&](uint32_t q) -> bool {
       const uint32_t slot = q % NSLOT;
-      PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 15, q);)
       bool r_ok = q < (uint32_t)NSLOT ||
                   warp_wait(bar(C::B_EMPTY + slot), ((q / NSLOT) - 1) & 1, abort_flag, tmo);
       if (r_ok && lane == 0) {
@@ -262,7 +482,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       return r_ok;
     };
     auto own_barrier = [&](uint32_t q) -> bool { return rank == 0 || tail_fill(q); };
-    int32_t row_prev = a.oob_row, row_cur = pre_row0, row_next = pre_row1;
+    uint32_t issued_end = 0;
+    // K half tile m (keys 64*rank..+63 of tile m, all of D): slot k holds panels 2k, 2k+1
+    auto issue_k = [&](int m, int32_t rows) {
+      const uint32_t item = pair_k_item(m);
+      for (int k = 0; k < 2 && ok; ++k) {
+        const uint32_t q = item * 2 + k;
+        const int l = lane, pl = l / k_per_panel, sub = l - pl * k_per_panel;
+        const int32_t row = key_row(rows, 64 * (int)rank + sub * k_rows);
+        if ((int)(q % kPairIssuers) != w) continue;
+        if (!(ok = acquire(q))) break;
+        const uint32_t sl = q % NSLOT;
+        if (l < 2 * k_per_panel) {
+          const uint32_t dst = slot_addr(sl) + pl * (kPanel / 2) + sub * k_rows * 128;
+          if (own_barrier(q))
+            tma_load_3d(dst, &tm_k, bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
+          else
+            tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
+        }
+        issued_end = q + 1;
+        PA_UNIT_ONLY(if (q == 0 && lane == 0 && blockIdx.x < 8192)
+                         g_pa_units[kUnitWords * blockIdx.x + 11] = clock64();)
+      }
+    };
+    // V half tile j (dims 128*rank..+127 of tile j): slot k holds keys 64k..64k+63
+    auto issue_v = [&](int j, int32_t rows) {
+      const uint32_t item = pair_v_item(j, n);
+      for (int k = 0; k < 2 && ok; ++k) {
+        const uint32_t q = item * 2 + k;
+        const int32_t row = key_row(rows, 64 * k + lane * v_rows);
+        if ((int)(q % kPairIssuers) != w) continue;
+        if (!(ok = acquire(q))) break;
+        const uint32_t sl = q % NSLOT;
+        if (lane < v_per_slot) {
+          const uint32_t dst = slot_addr(sl) + lane * (v_rows * 256);
+          if (own_barrier(q))
+            tma_load_4d(dst, &tm_v, bar(C::B_FULL + sl), 0, row, 2 * (int)rank, g);
+          else
+            tma_load_4d_pair(dst, &tm_v, leader_bar(C::B_FULL + sl), 0, row, 2 * (int)rank, g);
+        }
+        issued_end = q + 1;
+      }
+    };
     // Q tile: four 16 KB panels of 128/G whole tokens; both CTAs' bytes complete on rank 0's
     // barrier, which rank 0 arms for both. Rows past the piece arrive as zeros.
     if (a.q_tma && w == 0 && lane == 0) {
@@ -276,169 +537,114 @@ __global__ void __launch_bounds__(kThreads, 1)
                            g, t0);
       }
     }
-    uint32_t issued_end = 0;
-    for (int j = 0; j <= n && ok; ++j) {
-      if (j < n) {  // K half tile j: slot k holds panels 2k, 2k+1 of keys 64*rank..+63
-        const uint32_t item = j == 0 ? 0u : 2u * j - 1u;
-        for (int k = 0; k < 2 && ok; ++k) {
-          const uint32_t q = item * 2 + k;
-          const int l = lane, pl = l / k_per_panel, sub = l - pl * k_per_panel;
-          const int32_t row = key_row(row_cur, 64 * (int)rank + sub * k_rows);
-          if ((int)(q % kIssuers) != w) continue;
-          if (!(ok = acquire(q))) break;
-          const uint32_t slot = q % NSLOT;
-          if (l < 2 * k_per_panel) {
-            const uint32_t dst = slot_addr(slot) + pl * (kPanel / 2) + sub * k_rows * 128;
-            if (own_barrier(q))
-              tma_load_3d(dst, &tm_k, bar(C::B_FULL + slot), (2 * k + pl) * 64, g, row);
-            else
-              tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + slot), (2 * k + pl) * 64, g,
-                               row);
-          }
-          issued_end = q + 1;
-          PA_UNIT_ONLY(if (q == 0 && lane == 0 && blockIdx.x < 8192)
-                           g_pa_units[kUnitWords * blockIdx.x + 11] = clock64();)
-          PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 1, q);)
-        }
-      }
-      if (ok && j >= 1) {  // V half tile j-1: slot k holds keys 64k..64k+63, dims 128*rank..+127
-        const uint32_t item = v_item(j - 1, n);
-        for (int k = 0; k < 2 && ok; ++k) {
-          const uint32_t q = item * 2 + k;
-          const int32_t row = key_row(row_prev, 64 * k + lane * v_rows);
-          if ((int)(q % kIssuers) != w) continue;
-          if (!(ok = acquire(q))) break;
-          const uint32_t slot = q % NSLOT;
-          if (lane < v_per_slot) {
-            const uint32_t dst = slot_addr(slot) + lane * (v_rows * 256);
-            if (own_barrier(q))
-              tma_load_4d(dst, &tm_v, bar(C::B_FULL + slot), 0, row, 2 * (int)rank, g);
-            else
-              tma_load_4d_pair(dst, &tm_v, leader_bar(C::B_FULL + slot), 0, row, 2 * (int)rank,
-                               g);
-          }
-          issued_end = q + 1;
-          PA_TRACE_ONLY(if (lane == 0) tlog(w, tln, 2, q);)
-        }
-      }
-      row_prev = row_cur;
-      row_cur = row_next;
-      row_next = fetch(j + 2);
+    // Page rows of tiles j .. j+4 (lane i: page i of the tile). Iteration j issues K(j+2) and
+    // V(j) and loads the rows of tile j+5, which the K copy of iteration j+3 first uses: the
+    // page-table load has three iterations to land instead of stalling the next one.
+    int32_t row_j = pre_row0, row_j1 = pre_row1;
+    int32_t row_j2 = fetch(2), row_j3 = fetch(3), row_j4 = fetch(4);
+    issue_k(0, row_j);
+    if (n > 1 && ok) issue_k(1, row_j1);
+    for (int j = 0; j < n && ok; ++j) {
+      if (j + 2 < n) issue_k(j + 2, row_j2);
+      if (ok) issue_v(j, row_j);
+      row_j = row_j1;
+      row_j1 = row_j2;
+      row_j2 = row_j3;
+      row_j3 = row_j4;
+      row_j4 = fetch(j + 5);
     }
-    // Wait for this warp's copies among the last NSLOT fills (see the single-CTA kernel). On
-    // rank 0 the barrier covers both halves, so rank 1's copies have landed as well; rank 1
-    // drains only the tail fills on its own barrier, and it stays resident until rank 0 has
-    // finished (teardown handshake below).
+    // Wait for this warp's copies among the last NSLOT fills. On rank 0 the barrier covers both
+    // halves, so rank 1's copies have landed as well; rank 1 drains only the tail fills on its
+    // own barrier, and it stays resident until rank 0 has finished (teardown handshake below).
     const uint32_t all_fills = 4u * n;
     for (uint32_t q = all_fills > (uint32_t)NSLOT ? all_fills - NSLOT : 0; q < issued_end; ++q)
-      if ((int)(q % kIssuers) == w && own_barrier(q))
+      if ((int)(q % kPairIssuers) == w && own_barrier(q))
         drain_wait(bar(C::B_FULL + q % NSLOT), rank == 0 ? (q / NSLOT) & 1 : 0u, abort_flag,
                    tmo);
     __syncwarp();
   } else if (rank == 0) {
-    // ============================================================ MMA issuer (rank 0, one lane)
+    // ============================================================ MMA issuers (rank 0)
+    // warp 4 lane 0 issues every QK, warp 7 lane 0 every PV; each commits only its own MMAs
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_f16(256, kTileKeys, BF16, false);
       constexpr uint32_t idesc_pv = umma_idesc_f16(256, D, BF16, true);
       constexpr uint32_t kSlotDesc = kPanel >> 4;
       constexpr uint16_t kBoth = 0x3;
-      const uint64_t q_desc = smem_desc_sw128(sb + C::Q_OFF, 16, 1024);
-      const uint64_t k_desc = smem_desc_sw128(sb + C::RING_OFF, 16, 1024);
-      const uint64_t v_desc =
-          smem_desc_sw128(sb + C::RING_OFF, (uint32_t)(1 << a.v_shift) * 128u, 1024);
-      uint32_t slot = 0, round = 0;
-      PA_TRACE_ONLY(unsigned tln_w = 0;)
-      // a slot is ready when both halves landed (one barrier; for the tail fills rank 1's half
-      // is covered by its softmax warps' P-ready arrival, which waits for it)
-      PA_UNIT_ONLY(long long w_k = 0, w_v = 0, w_p = 0; long long* w_sel = &w_k;)
-      auto wait_slot = [&]() -> bool {
-        PA_TRACE_ONLY(tlog(6, tln_w, 11, round * NSLOT + slot);)
-        PA_UNIT_ONLY(const long long c0 = clock64();)
-        const bool r = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
-        PA_UNIT_ONLY(*w_sel += clock64() - c0;)
-        PA_TRACE_ONLY(tlog(6, tln_w, 12, round * NSLOT + slot);)
-        return r;
+      // fill q of the ring: slot q % NSLOT, landed when phase (q / NSLOT) % 2 of its barrier
+      // completes (one barrier for both halves; for the tail fills rank 1's half is covered by
+      // its softmax warps' P arrival, which they give after waiting for it)
+      auto wait_fill = [&](uint32_t q) -> bool {
+        return thread_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1u, abort_flag, tmo);
       };
-      auto advance = [&]() {
-        if (++slot == (uint32_t)NSLOT) {
-          slot = 0;
-          ++round;
-        }
-      };
-      bool ok = wait_cluster(bar(C::B_QFULL), 0);
-      PA_UNIT_ONLY(if (blockIdx.x < 8192) g_pa_units[kUnitWords * blockIdx.x + 8] = clock64();)
-      tc_fence_after();
-      for (int j = 0; j <= n && ok; ++j) {
-        if (j < n) {
-          const uint32_t s_tmem = tmem + kSCol0 + 128u * (j & 1);
+      bool ok = true;
+      if (warp == kMmaWarp) {
+        const uint64_t q_desc = smem_desc_sw128(sb + C::Q_OFF, 16, 1024);
+        const uint64_t k_desc = smem_desc_sw128(sb + C::RING_OFF, 16, 1024);
+        const uint32_t s_tmem = tmem + kPairSCol;
+        // S(m) = Q K(m)^T into the S buffer once the softmax has read S(m-1): slot k of the K
+        // half tile holds D panels 2k and 2k+1 (Q panels 2k, 2k+1). S(m) is completion m of
+        // s_full and the read of S(m) arrival m of s_free.
+        ok = wait_cluster(bar(C::B_QFULL), 0);
+        PA_UNIT_ONLY(if (blockIdx.x < 8192) g_pa_units[kUnitWords * blockIdx.x + 8] = clock64();)
+        for (int m = 0; m < n && ok; ++m) {
+          if (m >= 1) ok = wait_cluster(bar(C::B_SFREE), (uint32_t)(m - 1) & 1u);
+          const uint32_t q0 = 2u * pair_k_item(m);
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            PA_UNIT_ONLY(w_sel = &w_k;)
-            if (!(ok = wait_slot())) break;
-            PA_UNIT_ONLY(if (j == 0 && k == 0 && blockIdx.x < 8192)
+          for (int k = 0; k < 2 && ok; ++k) {
+            if (!(ok = wait_fill(q0 + k))) break;
+            PA_UNIT_ONLY(if (m == 0 && k == 0 && blockIdx.x < 8192)
                              g_pa_units[kUnitWords * blockIdx.x + 9] = clock64();)
-            PA_TRACE_ONLY(tlog(3, tln, 3, round * NSLOT + slot);)
             tc_fence_after();
+            const uint32_t sl = (q0 + k) % NSLOT;
 #pragma unroll
             for (int pl = 0; pl < 2; ++pl) {
               const int p = 2 * k + pl;
               const uint64_t ad = q_desc + p * kSlotDesc;
-              const uint64_t bd = k_desc + slot * kSlotDesc + pl * (kSlotDesc / 2);
-              umma_ss_pair(s_tmem, ad, bd, idesc_qk, p != 0 ? 1u : 0u);
-              umma_ss_pair(s_tmem, ad + 2, bd + 2, idesc_qk, 1u);
-              umma_ss_pair(s_tmem, ad + 4, bd + 4, idesc_qk, 1u);
-              umma_ss_pair(s_tmem, ad + 6, bd + 6, idesc_qk, 1u);
-            }
-            umma_commit_pair(bar(C::B_EMPTY + slot), kBoth);
-            PA_TRACE_ONLY(tlog(3, tln, 4, round * NSLOT + slot);)
-            advance();
-          }
-          if (!ok) break;
-          umma_commit_pair(bar(C::B_SFULL + (j & 1)), kBoth);
-        }
-        if (j >= 1) {
-          const int i = j - 1;
-          PA_TRACE_ONLY(tlog(6, tln_w, 14, i);)
-          PA_UNIT_ONLY(const long long c0 = clock64();)
-          ok = wait_cluster(bar(C::B_PFULL + (i & 1)), (i >> 1) & 1);
-          PA_UNIT_ONLY(w_p += clock64() - c0; w_sel = &w_v;)
-          PA_TRACE_ONLY(tlog(3, tln, 5, i);)
-          // Each half of the V tile (keys 0-63, then 64-127) is multiplied as soon as its slot
-          // has landed, and its slot is released right after its four MMAs.
-          const uint32_t p_tmem = tmem + kSCol0 + 128u * (i & 1) + kPColOff;
+              const uint64_t bd = k_desc + sl * kSlotDesc + pl * (kSlotDesc / 2);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (ok) ok = wait_slot();
-            if (!ok) break;
+              for (int ks = 0; ks < 4; ++ks)
+                umma_ss_pair(s_tmem, ad + 2 * ks, bd + 2 * ks, idesc_qk, (p | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(bar(C::B_EMPTY + sl), kBoth);
+          }
+          if (ok) umma_commit_pair(bar(C::B_SFULL), kBoth);
+        }
+      } else {
+        const uint64_t v_desc =
+            smem_desc_sw128(sb + C::RING_OFF, (uint32_t)(1 << a.v_shift) * 128u, 1024);
+        // O += P(i) V(i) once P(i) is stored (phase (i / 2) % 2 of p_full[i % 2]): each half of
+        // the V tile (keys 0-63, then 64-127) against the matching columns of P(i)'s buffer
+        // (16 keys = 8 columns), released after its 4 MMAs; PV(i) completes phase (i / 2) % 2
+        // of pv_done[i % 2]
+        for (int i = 0; i < n && ok; ++i) {
+          ok = wait_cluster(bar(C::B_PFULL + (i & 1)), (uint32_t)(i >> 1) & 1u);
+          const uint32_t p_tmem = tmem + kPairPCol + 64u * (uint32_t)(i & 1);
+          const uint32_t q0 = 2u * pair_v_item(i, n);
+#pragma unroll
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (!(ok = wait_fill(q0 + h))) break;
             tc_fence_after();
+            const uint32_t sl = (q0 + h) % NSLOT;
 #pragma unroll
             for (int ks = 4 * h; ks < 4 * h + 4; ++ks) {
               const uint32_t off = v_offset_pair(16u * ks, 0, a.v_shift);
-              umma_ts_pair(tmem + kOCol, p_tmem + ks * 8,
-                           v_desc + slot * kSlotDesc + ((off & (kPanel - 1)) >> 4), idesc_pv,
+              umma_ts_pair(tmem + kOCol, p_tmem + (uint32_t)ks * 8u,
+                           v_desc + sl * kSlotDesc + ((off & (kPanel - 1)) >> 4), idesc_pv,
                            (i > 0 || ks > 0) ? 1u : 0u);
             }
-            umma_commit_pair(bar(C::B_EMPTY + slot), kBoth);
-            advance();
+            umma_commit_pair(bar(C::B_EMPTY + sl), kBoth);
           }
-          if (!ok) break;
-          PA_TRACE_ONLY(tlog(3, tln, 6, round * NSLOT + slot - 2);)
-          umma_commit_pair(bar(C::B_PVDONE + (i & 1)), kBoth);
-          PA_TRACE_ONLY(tlog(3, tln, 7, i);)
+          if (ok) umma_commit_pair(bar(C::B_PVDONE + (i & 1)), kBoth);
         }
       }
-      PA_UNIT_ONLY(if (blockIdx.x < 8192) {
-        g_pa_units[kUnitWords * blockIdx.x + 12] = (unsigned long long)w_k;
-        g_pa_units[kUnitWords * blockIdx.x + 13] = (unsigned long long)w_v;
-        g_pa_units[kUnitWords * blockIdx.x + 14] = (unsigned long long)w_p;
-      })
+      // every MMA of both issuers must finish before tensor memory is freed
       umma_commit_pair(bar(C::B_MMADONE), kBoth);
       drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
     }
     __syncwarp();
   } else {
-    // ============================================================ rank 1, MMA warp
-    // rank 0's last MMA has read this CTA's shared and tensor memory
+    // ============================================================ rank 1, MMA warps
+    // rank 0's last MMAs have read this CTA's shared and tensor memory
     if (lane == 0) drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
     __syncwarp();
   }
