@@ -40,6 +40,10 @@ struct CostModel {
   }
 };
 
+// K/V bytes of a piece above which the row blocks of a head are scheduled as teams (about
+// three quarters of the 126 MB L2).
+constexpr double kTeamKvBytes = 96e6;
+
 // CTAs per unit: head dim 256 runs on CTA pairs (two Q tiles share each K/V tile load).
 int ctas_per_unit_for(int D) { return D == 256 ? 2 : 1; }
 
@@ -96,25 +100,27 @@ double simulate_items(const std::vector<pa::PaItem>& items, int slots, const Cos
 
 namespace pa {
 
-// McNaughton's wrap-around rule over the row blocks' KV tiles: lay the row blocks end to end
-// (longest first), fill `slots` workers to an equal load in turn, and cut a row block where a
-// worker's share ends. Every worker then carries the same load and at most one cut per worker
-// boundary is made; no piece shorter than `m` tiles is cut off. Items are issued in the order of
-// their planned start, so the hardware's first-free-SM dispatch reproduces the plan.
-// len[rb] is the KV-tile count of row block rb; `order` lists the row blocks longest first.
-static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32_t>& order,
-                        int slots, int per, int head_dim, Schedule* out) {
-  const CostModel cm(head_dim);
-  const int64_t n_rb = (int64_t)len.size();
-  if (n_rb > kMaxItems || n_rb == 0) return false;
+// McNaughton's wrap-around rule: lay the runs of KV tiles (lengths len[order[0]], ...) end to
+// end, fill `workers` to an equal load in turn, and cut a run where a worker's share ends.
+// Every worker then carries the same load and at most one cut per worker boundary is made; no
+// piece shorter than `m` tiles is cut off, and no run is cut into more parts than the combine
+// merges. Returns the pieces (run, first tile, end tile, worker, planned start).
+struct Piece {
+  int32_t rb, kt0, kt1, worker;
+  double start;
+};
+
+static bool wrap_cut(const std::vector<int64_t>& len, const std::vector<int32_t>& order,
+                     int workers, double c_item, std::vector<Piece>* out) {
+  const int64_t n = (int64_t)order.size();
+  if (n == 0 || workers <= 0) return false;
   double total = 0.0;
-  for (int64_t x : len) total += (double)x;
-  const double c_item = cm.unit_us / cm.tile_us;  // fixed cost of an item, in tiles
-  struct Piece {
-    int32_t rb, kt0, kt1, worker;
-    double start;
-  };
-  std::vector<Piece> pieces;
+  int64_t max_len = 0;
+  for (int32_t r : order) {
+    total += (double)len[r];
+    max_len = std::max(max_len, len[r]);
+  }
+  std::vector<Piece>& pieces = *out;
   // Wrap-around assignment for a given share per worker; returns the workers it needs.
   auto assign = [&](double share, int64_t m, double over) -> int {
     pieces.clear();
@@ -130,7 +136,7 @@ static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32
         } else if (load > 0.0 && room < (double)m) {
           ++k;       // this worker is full
           load = 0.0;
-          if (k > slots) return k + 1;  // cannot fit: stop early
+          if (k > workers) return k + 1;  // cannot fit: stop early
           continue;
         } else {
           // at least m tiles (a fresh worker always makes progress), and leave at least m
@@ -149,18 +155,23 @@ static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32
     }
     return k + 1;
   };
-  // The smallest share (from the even split of the tiles plus one item cost per row block and
-  // per cut) whose assignment fits the workers.
-  double share = (total + c_item * (double)(n_rb + slots - 1)) / slots;
-  // no row block in more parts than the combine merges (a part may also start and end a worker
-  // part-way, hence one part of slack)
-  int64_t max_len = 0;
-  for (int64_t x : len) max_len = std::max(max_len, x);
+  // The smallest share (from the even split of the tiles plus one item cost per run and per
+  // cut) whose assignment fits the workers; no run in more parts than the combine merges (a
+  // part may also start and end a worker part-way, hence one part of slack).
+  double share = (total + c_item * (double)(n + workers - 1)) / workers;
   share = std::max(share, (double)max_len / (PA_MAX_SPLITS - 2) + c_item + 1.0);
   const int64_t m = std::max<int64_t>(4, (int64_t)(share / 32.0));
   const double over = 1.0 + share / 128.0;
-  for (int it = 0; it < 400 && assign(share, m, over) > slots; ++it) share *= 1.002;
-  if (assign(share, m, over) > slots) return false;
+  for (int it = 0; it < 400 && assign(share, m, over) > workers; ++it) share *= 1.002;
+  return assign(share, m, over) <= workers;
+}
+
+// The schedule of a set of pieces of the row blocks (numbered 0 .. n_rb-1): workspace slots
+// for the parts of cut row blocks, items in the order of their planned start (so that the
+// hardware's first-free dispatch reproduces the plan), and the simulated makespan.
+static bool finish_schedule(const std::vector<Piece>& pieces, int64_t n_rb, int slots, int per,
+                            int head_dim, Schedule* out) {
+  const CostModel cm(head_dim);
   if ((int64_t)pieces.size() > kMaxItems) return false;
   // workspace slots: consecutive for the parts of each cut row block, in row-block order
   std::vector<int32_t> parts(n_rb, 0);
@@ -177,11 +188,20 @@ static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32
     sch.max_parts = std::max(sch.max_parts, parts[rb]);
   }
   if ((int64_t)sch.split.size() > kMaxSplitBlocks || sch.max_parts > PA_MAX_SPLITS) return false;
+  // the parts of a row block take its slots in key order
+  std::vector<const Piece*> by_key;
+  for (const Piece& pc : pieces) by_key.push_back(&pc);
+  std::stable_sort(by_key.begin(), by_key.end(), [](const Piece* x, const Piece* y) {
+    return x->rb != y->rb ? x->rb < y->rb : x->kt0 < y->kt0;
+  });
+  std::vector<int32_t> slot_of(pieces.size(), -1);
   std::vector<int32_t> seen(n_rb, 0);
+  for (const Piece* pc : by_key)
+    if (parts[pc->rb] > 1) slot_of[pc - pieces.data()] = first[pc->rb] + seen[pc->rb]++;
   std::vector<std::pair<std::pair<double, int>, PaItem>> items;
-  for (const Piece& pc : pieces) {  // pieces of a row block appear in key order
-    const int32_t slot = parts[pc.rb] > 1 ? first[pc.rb] + seen[pc.rb]++ : -1;
-    items.push_back({{pc.start, pc.worker}, PaItem{pc.rb, pc.kt0, pc.kt1, slot}});
+  for (size_t i = 0; i < pieces.size(); ++i) {
+    const Piece& pc = pieces[i];
+    items.push_back({{pc.start, pc.worker}, PaItem{pc.rb, pc.kt0, pc.kt1, slot_of[i]}});
   }
   std::stable_sort(items.begin(), items.end(),
                    [](const auto& x, const auto& y) { return x.first < y.first; });
@@ -198,23 +218,103 @@ static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32
   return true;
 }
 
-bool build_balanced(const pa_plan_t& p, Schedule* out) {
-  const int per = ctas_per_unit_for(p.head_dim);
-  const int slots = std::max(1, p.num_sms / per);
-  const int64_t q_units = ((int64_t)p.q_tiles + per - 1) / per;
-  const int Hkv = p.n_kv_heads;
+// The wrap-around rule over whole row blocks, one worker (SM or SM pair) each.
+static bool wrap_around(const std::vector<int64_t>& len, const std::vector<int32_t>& order,
+                        int slots, int per, int head_dim, Schedule* out) {
+  const CostModel cm(head_dim);
+  const int64_t n_rb = (int64_t)len.size();
+  if (n_rb > kMaxItems || n_rb == 0) return false;
+  std::vector<Piece> pieces;
+  if (!wrap_cut(len, order, slots, cm.unit_us / cm.tile_us, &pieces)) return false;
+  return finish_schedule(pieces, n_rb, slots, per, head_dim, out);
+}
+
+// The wrap-around rule over teams: `bundles` are groups of row blocks that read the same KV
+// head (longest first within a group); a team of t = bundle size workers runs a bundle piece
+// [a, b) as one item per row block, all starting together, so the team streams each K/V tile
+// of the head at the same time and L2 serves its repeated reads. `slots` / t teams; a bundle's
+// length is its longest row block's, and shorter ones end their last piece early.
+static bool wrap_teams(const std::vector<int64_t>& len,
+                       const std::vector<std::vector<int32_t>>& bundles, int t, int slots,
+                       int per, int head_dim, Schedule* out) {
+  const CostModel cm(head_dim);
+  const int64_t n_rb = (int64_t)len.size();
+  const int teams = slots / t;
+  if (teams < 1 || bundles.empty()) return false;
+  std::vector<int64_t> blen(bundles.size());
+  std::vector<int32_t> border(bundles.size());
+  for (size_t b = 0; b < bundles.size(); ++b) {
+    int64_t mx = 0;
+    for (int32_t rb : bundles[b]) mx = std::max(mx, len[rb]);
+    blen[b] = mx;
+    border[b] = (int32_t)b;
+  }
+  std::vector<Piece> team_pieces;
+  if (!wrap_cut(blen, border, teams, cm.unit_us / cm.tile_us, &team_pieces)) return false;
+  std::vector<Piece> pieces;
+  for (const Piece& tp : team_pieces) {
+    const std::vector<int32_t>& members = bundles[tp.rb];
+    for (size_t i = 0; i < members.size(); ++i) {
+      const int32_t rb = members[i];
+      if (tp.kt0 >= len[rb]) continue;
+      pieces.push_back({rb, tp.kt0, (int32_t)std::min<int64_t>(tp.kt1, len[rb]),
+                        tp.worker * t + (int32_t)i, tp.start});
+    }
+  }
+  return finish_schedule(pieces, n_rb, slots, per, head_dim, out);
+}
+
+// The balanced schedule of one piece (R rows at history H) of q_units row blocks a KV head.
+static bool balanced_piece(int64_t q_tiles, int64_t R, int64_t H, int G, int Hkv, int head_dim,
+                           int num_sms, Schedule* out) {
+  const int per = ctas_per_unit_for(head_dim);
+  const int slots = std::max(1, num_sms / per);
+  const int64_t q_units = (q_tiles + per - 1) / per;
   const int64_t n_rb = q_units * Hkv;
   if (n_rb > kMaxItems || n_rb <= 0) return false;
   std::vector<int64_t> len(n_rb);
-  std::vector<int32_t> order(n_rb);
-  for (int64_t rb = 0; rb < n_rb; ++rb) {  // row-block numbering is already longest first
+  std::vector<int32_t> order;
+  order.reserve(n_rb);
+  for (int64_t rb = 0; rb < n_rb; ++rb) {
     int64_t qu;
     int g;
     rb_coords((int32_t)rb, q_units, Hkv, &qu, &g);
-    len[rb] = unit_kv_tiles(qu, per, p.q_tiles, p.chunk_rows, p.group, p.hist_len);
-    order[rb] = (int32_t)rb;
+    len[rb] = unit_kv_tiles(qu, per, q_tiles, R, G, H);
   }
-  return wrap_around(len, order, slots, per, p.head_dim, out);
+  // The row blocks of one KV head one after another, longest first within the head (which
+  // the numbering rb = g, g + Hkv, ... already is).
+  for (int g = 0; g < Hkv; ++g)
+    for (int64_t rb = g; rb < n_rb; rb += Hkv) order.push_back((int32_t)rb);
+  // When the piece's K/V do not fit in L2, every row block of a head reads all of the head's
+  // keys from HBM unless the row blocks stream them together: measured on a 128-row piece at
+  // 131,072 keys (3 row blocks a head) 3.0x the K/V bytes from HBM, and on a 512-row piece at
+  // 34K keys (12 a head) 10x. Then the row blocks of a head run as teams (wrap_teams) of t
+  // workers, t as large as leaves at most a tenth of the workers idle.
+  const double kv_bytes = 2.0 * (double)(H + R) * Hkv * head_dim * 2.0;
+  const int64_t k = q_units;  // row blocks a head
+  if (kv_bytes > kTeamKvBytes && k >= 2) {
+    for (int64_t r = 1; r <= k; ++r) {
+      const int t = (int)ceil_div64(k, r);
+      const int teams = slots / t;
+      if (teams < 1 || slots - teams * t > slots / 10) continue;
+      std::vector<std::vector<int32_t>> bundles;
+      for (int g = 0; g < Hkv; ++g)
+        for (int64_t i = 0; i < k; i += t) {
+          std::vector<int32_t> b;
+          for (int64_t j = i; j < std::min<int64_t>(k, i + t); ++j)
+            b.push_back((int32_t)(g + j * Hkv));
+          bundles.push_back(std::move(b));
+        }
+      if (wrap_teams(len, bundles, t, slots, per, head_dim, out)) return true;
+      break;
+    }
+  }
+  return wrap_around(len, order, slots, per, head_dim, out);
+}
+
+bool build_balanced(const pa_plan_t& p, Schedule* out) {
+  return balanced_piece(p.q_tiles, p.chunk_rows, p.hist_len, p.group, p.n_kv_heads, p.head_dim,
+                        p.num_sms, out);
 }
 
 int describe_batch(int batch, const int32_t* q_lens, const int64_t* hist_lens, int G, int Hkv,
@@ -247,6 +347,10 @@ int batch_ctas_per_unit(int head_dim, int G, int batch, const int32_t* q_lens) {
 
 bool build_batch(int num_sms, int head_dim, int per, int G, int Hkv, const Batch& bt,
                  Schedule* out) {
+  // one sequence: the single piece's schedule (row blocks numbered the same way)
+  if (bt.seq.size() == 1 && per == ctas_per_unit_for(head_dim))
+    return balanced_piece(q_tiles_for(bt.seq[0].rows, G), bt.seq[0].rows, bt.seq[0].hist, G,
+                          Hkv, head_dim, num_sms, out);
   const int slots = std::max(1, num_sms / per);
   std::vector<int64_t> len;
   for (const PaSeq& sq : bt.seq) {
