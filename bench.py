@@ -36,7 +36,11 @@ L2_FLUSH_BYTES = 512 << 20
 # combined over the 16 chunks as stated in "chunks" and "how"). It stands for the kernel whose
 # sources hash to `sources`; after any change to them the bench reports null until the
 # captures are taken again.
-TRAFFIC_CAPTURE = None
+TRAFFIC_CAPTURE = {
+    "workload": "c5", "sources": "da9b3e89bea657f7", "bytes_per_launch": 111.16e6,
+    "how": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch each of chunks 0, 3, "
+            "6, 9, 12 and 15 (21.2, 39.4, 64.4, 95.3, 154.3, 337.9 MB; three launches per capture "
+            "of bench.py --section piece), linear in between, mean over the 16 chunks")}
 
 
 def kernel_sources_hash() -> str:
