@@ -22,9 +22,11 @@
 // tcgen05.mma holds its issuing thread until the tensor pipe takes the instruction, so a
 // single issuer leaves the pipe idle through every wait and commit between its MMA groups
 // (measured: ~900 of ~3,100 cycles per tile); with two, one stream feeds the pipe while the
-// other waits, and QK and PV (different accumulators) interleave. Copies land in a ring of
-// ten 16 KB slots in the order K0, K1, then per tile j, K(j+2) and V(j); each issuer finds its
-// slots from these positions.
+// other waits, and QK and PV (different accumulators) interleave. K and V land in rings of
+// their own (three and two half tiles of 16 KB slots), each filled in tile order by a copy warp
+// of its own: V(j) reuses the slots of V(j-2) (released when PV(j-2) completes), not those
+// of a K half tile that QK(j) releases just before PV(j) needs V(j), which left V one tile
+// of lookahead and made small pages (more boxes to issue per tile) land late.
 //
 // Rank 1's softmax warps announce the end of their S reads and their P to rank 0 with
 // CTA-scope remote arrivals (tensor-memory accesses, ordered by tcgen05.wait and the
@@ -44,12 +46,14 @@ constexpr uint32_t kPairPCol = 384;  // P: buffers of 64 columns (16-bit pairs) 
 
 struct PairCfg {
   static constexpr int NP = 4;        // 64-wide panels of a 256-wide row
-  static constexpr int NSLOT = 10;    // ring of 16 KB slots; a half tile (K or V) is 2 slots
+  static constexpr int KSLOT = 6;     // K ring: 16 KB slots, a half tile is 2 slots
+  static constexpr int VSLOT = 4;     // V ring (after the K ring)
+  static constexpr int NSLOT = KSLOT + VSLOT;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NP * kPanel;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * kPanel;
-  // full[10] (rank 0: both halves landed), empty[10], q_full, s_full, s_free, p_full[2],
-  // pv_done[2], mma_done (both issuers' last commits), teardown
+  // full[10] (rank 0: both halves landed), empty[10] (K ring slots 0-5, V ring 6-9), q_full,
+  // s_full, s_free, p_full[2], pv_done[2], mma_done (both issuers' last commits), teardown
   static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_QFULL = 2 * NSLOT,
                        B_SFULL = 2 * NSLOT + 1, B_SFREE = 2 * NSLOT + 2, B_PFULL = 2 * NSLOT + 3,
                        B_PVDONE = 2 * NSLOT + 5, B_MMADONE = 2 * NSLOT + 7,
@@ -70,12 +74,15 @@ __device__ __forceinline__ uint32_t v_offset_pair(uint32_t k, uint32_t pl, int v
          ((kk & ((1u << v_shift) - 1u)) << 7);
 }
 
-// Positions of the half tiles in the ring's fill order K0, K1, then per tile j: K(j+2) (while
-// j + 2 < n), V(j). K tile m and V tile j of a unit of n tiles:
-__device__ __forceinline__ uint32_t pair_k_item(int m) { return m <= 1 ? (uint32_t)m : 2u * m - 2u; }
-__device__ __forceinline__ uint32_t pair_v_item(int j, int n) {
-  return j <= n - 3 ? 2u * j + 3u : (j == n - 2 ? 2u * n - 2u : 2u * n - 1u);
+// Fill q of a ring (half tile q / 2, slot half q % 2): K fill q sits in slot q % KSLOT, V fill
+// q in slot KSLOT + q % VSLOT; a fill has landed when phase (q / ring size) % 2 of its slot's
+// full barrier completes.
+__device__ __forceinline__ uint32_t pair_k_slot(uint32_t q) { return q % PairCfg::KSLOT; }
+__device__ __forceinline__ uint32_t pair_k_phase(uint32_t q) { return (q / PairCfg::KSLOT) & 1u; }
+__device__ __forceinline__ uint32_t pair_v_slot(uint32_t q) {
+  return PairCfg::KSLOT + q % PairCfg::VSLOT;
 }
+__device__ __forceinline__ uint32_t pair_v_phase(uint32_t q) { return (q / PairCfg::VSLOT) & 1u; }
 
 // Barriers of the pair's softmax warps besides those of SoftmaxCtx.
 struct PairSync {
@@ -329,9 +336,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   auto leader_bar = [&](int i) -> uint32_t { return leader_bar0 + 8u * (uint32_t)i; };
   // The sequence's last KV tile, partly past the end (paged pools only: there the rows after
   // the last key hold another sequence's data or nothing), is the unit's last tile; its V
-  // fills are the unit's last two (4n-2, 4n-1).
+  // fills are the V ring's last two (2n-2, 2n-1).
   const bool has_tail = PAGED && (kt0 + n) * kTileKeys > a.total_keys;
-  auto tail_fill = [&](uint32_t q) -> bool { return has_tail && q + 2u >= 4u * (uint32_t)n; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSLOT; ++i) {
@@ -417,15 +423,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // Those fills complete on this CTA's own barrier: on rank 1 that barrier sees no other
     // phase, so its parity is 0.
     auto v_tail = [&](int j, int r) -> bool {
-      const uint32_t seq0 = pair_v_item(j, n) * 2;
+      const uint32_t seq0 = 2u * (uint32_t)j;
       bool okv = true;
       for (int k = 0; k < 2 && okv; ++k)
-        okv = warp_wait(bar(C::B_FULL + (seq0 + k) % NSLOT),
-                        rank == 0 ? ((seq0 + k) / NSLOT) & 1 : 0u, abort_flag, tmo);
+        okv = warp_wait(bar(C::B_FULL + pair_v_slot(seq0 + k)),
+                        rank == 0 ? pair_v_phase(seq0 + k) : 0u, abort_flag, tmo);
       if (!okv || r < 0) return okv;
       for (int pl = 0; pl < 2; ++pl) {
         const uint32_t off = v_offset_pair((uint32_t)r, pl, a.v_shift);
-        const uint32_t ra = slot_addr((seq0 + (off >> 14)) % NSLOT) + (off & (kPanel - 1));
+        const uint32_t ra = slot_addr(pair_v_slot(seq0 + (off >> 14))) + (off & (kPanel - 1));
 #pragma unroll
         for (int c = 0; c < 8; ++c) st_shared_v4(ra + c * 16, 0u, 0u, 0u, 0u);
       }
@@ -434,8 +440,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     softmax_pair_role<PAGED, BF16>(a, sc, ps, v_tail);
   } else if (warp > kMmaWarp && warp < kPairPvWarp) {
     // ============================================================ TMA issuers (two warps)
-    // Fill q (2 per K or V half tile, in the order of pair_k_item / pair_v_item) is issued by
-    // warp q % kPairIssuers; lanes issue one box each.
+    // Warp 5 fills the K ring (K(0), K(1), ... in tile order), warp 6 the V ring; lanes issue
+    // one box each.
     const int w = warp - kMmaWarp - 1;
     const int ppt = a.pages_per_tile;
     const int prow = a.page_rows;
@@ -467,61 +473,55 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const int32_t base = __shfl_sync(0xffffffffu, rows, pg & 31);
       return base == a.oob_row ? a.oob_row : base + (kk & (prow - 1));
     };
-    // Rank 0 expects both halves of a slot on its barrier; rank 1 arms its own barrier only for
-    // the tail fills.
-    auto acquire = [&](uint32_t q) -> bool {
-      const uint32_t slot = q % NSLOT;
-      bool r_ok = q < (uint32_t)NSLOT ||
-                  warp_wait(bar(C::B_EMPTY + slot), ((q / NSLOT) - 1) & 1, abort_flag, tmo);
+    // Wait until a slot is free for its `use`-th fill and announce the bytes. Rank 0 expects
+    // both halves of a slot on its barrier; rank 1 arms its own barrier only for the tail fills.
+    auto acquire = [&](uint32_t slot, uint32_t use, bool tail) -> bool {
+      bool r_ok =
+          use == 0 || warp_wait(bar(C::B_EMPTY + slot), (use - 1) & 1, abort_flag, tmo);
       if (r_ok && lane == 0) {
-        const bool tail = tail_fill(q);
         if (rank == 0) mbar_arrive_expect_tx(bar(C::B_FULL + slot), tail ? kPanel : 2 * kPanel);
         else if (tail) mbar_arrive_expect_tx(bar(C::B_FULL + slot), kPanel);
       }
       __syncwarp();
       return r_ok;
     };
-    auto own_barrier = [&](uint32_t q) -> bool { return rank == 0 || tail_fill(q); };
-    uint32_t issued_end = 0;
+    uint32_t issued = 0;  // fills this warp issued
     // K half tile m (keys 64*rank..+63 of tile m, all of D): slot k holds panels 2k, 2k+1
     auto issue_k = [&](int m, int32_t rows) {
-      const uint32_t item = pair_k_item(m);
       for (int k = 0; k < 2 && ok; ++k) {
-        const uint32_t q = item * 2 + k;
+        const uint32_t q = 2u * (uint32_t)m + (uint32_t)k;
         const int l = lane, pl = l / k_per_panel, sub = l - pl * k_per_panel;
         const int32_t row = key_row(rows, 64 * (int)rank + sub * k_rows);
-        if ((int)(q % kPairIssuers) != w) continue;
-        if (!(ok = acquire(q))) break;
-        const uint32_t sl = q % NSLOT;
+        const uint32_t sl = pair_k_slot(q);
+        if (!(ok = acquire(sl, q / C::KSLOT, false))) break;
         if (l < 2 * k_per_panel) {
           const uint32_t dst = slot_addr(sl) + pl * (kPanel / 2) + sub * k_rows * 128;
-          if (own_barrier(q))
+          if (rank == 0)
             tma_load_3d(dst, &tm_k, bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
           else
             tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
         }
-        issued_end = q + 1;
+        issued = q + 1;
         PA_UNIT_ONLY(if (q == 0 && lane == 0 && blockIdx.x < 8192)
                          g_pa_units[kUnitWords * blockIdx.x + 11] = clock64();)
       }
     };
     // V half tile j (dims 128*rank..+127 of tile j): slot k holds keys 64k..64k+63
     auto issue_v = [&](int j, int32_t rows) {
-      const uint32_t item = pair_v_item(j, n);
+      const bool tail = has_tail && j == n - 1;
       for (int k = 0; k < 2 && ok; ++k) {
-        const uint32_t q = item * 2 + k;
+        const uint32_t q = 2u * (uint32_t)j + (uint32_t)k;
         const int32_t row = key_row(rows, 64 * k + lane * v_rows);
-        if ((int)(q % kPairIssuers) != w) continue;
-        if (!(ok = acquire(q))) break;
-        const uint32_t sl = q % NSLOT;
+        const uint32_t sl = pair_v_slot(q);
+        if (!(ok = acquire(sl, q / C::VSLOT, tail))) break;
         if (lane < v_per_slot) {
           const uint32_t dst = slot_addr(sl) + lane * (v_rows * 256);
-          if (own_barrier(q))
+          if (rank == 0 || tail)
             tma_load_4d(dst, &tm_v, bar(C::B_FULL + sl), 0, row, 2 * (int)rank, g);
           else
             tma_load_4d_pair(dst, &tm_v, leader_bar(C::B_FULL + sl), 0, row, 2 * (int)rank, g);
         }
-        issued_end = q + 1;
+        issued = q + 1;
       }
     };
     // Q tile: four 16 KB panels of 128/G whole tokens; both CTAs' bytes complete on rank 0's
@@ -537,30 +537,30 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                            g, t0);
       }
     }
-    // Page rows of tiles j .. j+4 (lane i: page i of the tile). Iteration j issues K(j+2) and
-    // V(j) and loads the rows of tile j+5, which the K copy of iteration j+3 first uses: the
-    // page-table load has three iterations to land instead of stalling the next one.
-    int32_t row_j = pre_row0, row_j1 = pre_row1;
-    int32_t row_j2 = fetch(2), row_j3 = fetch(3), row_j4 = fetch(4);
-    issue_k(0, row_j);
-    if (n > 1 && ok) issue_k(1, row_j1);
-    for (int j = 0; j < n && ok; ++j) {
-      if (j + 2 < n) issue_k(j + 2, row_j2);
-      if (ok) issue_v(j, row_j);
-      row_j = row_j1;
-      row_j1 = row_j2;
-      row_j2 = row_j3;
-      row_j3 = row_j4;
-      row_j4 = fetch(j + 5);
+    // Page rows of tiles t .. t+3 (lane i: page i of the tile); the rows of tile t+4 are loaded
+    // while tile t is issued, three tiles before they are used.
+    int32_t row_0 = pre_row0, row_1 = pre_row1, row_2 = fetch(2), row_3 = fetch(3);
+    for (int t = 0; t < n && ok; ++t) {
+      if (w == 0)
+        issue_k(t, row_0);
+      else
+        issue_v(t, row_0);
+      row_0 = row_1;
+      row_1 = row_2;
+      row_2 = row_3;
+      row_3 = fetch(t + 4);
     }
-    // Wait for this warp's copies among the last NSLOT fills. On rank 0 the barrier covers both
-    // halves, so rank 1's copies have landed as well; rank 1 drains only the tail fills on its
-    // own barrier, and it stays resident until rank 0 has finished (teardown handshake below).
-    const uint32_t all_fills = 4u * n;
-    for (uint32_t q = all_fills > (uint32_t)NSLOT ? all_fills - NSLOT : 0; q < issued_end; ++q)
-      if ((int)(q % kPairIssuers) == w && own_barrier(q))
-        drain_wait(bar(C::B_FULL + q % NSLOT), rank == 0 ? (q / NSLOT) & 1 : 0u, abort_flag,
+    // Wait for this warp's last copies of each slot. On rank 0 the barrier covers both halves,
+    // so rank 1's copies have landed as well; rank 1 drains only the tail fills on its own
+    // barrier, and it stays resident until rank 0 has finished (teardown handshake below).
+    const uint32_t ring = w == 0 ? C::KSLOT : C::VSLOT;
+    for (uint32_t q = issued > ring ? issued - ring : 0; q < issued; ++q) {
+      const bool tail = w == 1 && has_tail && q + 2u >= 2u * (uint32_t)n;
+      if (rank == 0 || tail)
+        drain_wait(bar(C::B_FULL + (w == 0 ? pair_k_slot(q) : pair_v_slot(q))),
+                   rank == 0 ? (w == 0 ? pair_k_phase(q) : pair_v_phase(q)) : 0u, abort_flag,
                    tmo);
+    }
     __syncwarp();
   } else if (rank == 0) {
     // ============================================================ MMA issuers (rank 0)
@@ -570,11 +570,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       constexpr uint32_t idesc_pv = umma_idesc_f16(256, D, BF16, true);
       constexpr uint32_t kSlotDesc = kPanel >> 4;
       constexpr uint16_t kBoth = 0x3;
-      // fill q of the ring: slot q % NSLOT, landed when phase (q / NSLOT) % 2 of its barrier
-      // completes (one barrier for both halves; for the tail fills rank 1's half is covered by
-      // its softmax warps' P arrival, which they give after waiting for it)
-      auto wait_fill = [&](uint32_t q) -> bool {
-        return thread_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1u, abort_flag, tmo);
+      // a fill has landed (one barrier for both halves; for the tail fills rank 1's half is
+      // covered by its softmax warps' P arrival, which they give after waiting for it)
+      auto wait_fill = [&](uint32_t slot, uint32_t phase) -> bool {
+        return thread_wait(bar(C::B_FULL + slot), phase, abort_flag, tmo);
       };
       bool ok = true;
       if (warp == kMmaWarp) {
@@ -588,14 +587,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         PA_UNIT_ONLY(if (blockIdx.x < 8192) g_pa_units[kUnitWords * blockIdx.x + 8] = clock64();)
         for (int m = 0; m < n && ok; ++m) {
           if (m >= 1) ok = wait_cluster(bar(C::B_SFREE), (uint32_t)(m - 1) & 1u);
-          const uint32_t q0 = 2u * pair_k_item(m);
+          const uint32_t q0 = 2u * (uint32_t)m;
 #pragma unroll
           for (int k = 0; k < 2 && ok; ++k) {
-            if (!(ok = wait_fill(q0 + k))) break;
+            if (!(ok = wait_fill(pair_k_slot(q0 + k), pair_k_phase(q0 + k)))) break;
             PA_UNIT_ONLY(if (m == 0 && k == 0 && blockIdx.x < 8192)
                              g_pa_units[kUnitWords * blockIdx.x + 9] = clock64();)
             tc_fence_after();
-            const uint32_t sl = (q0 + k) % NSLOT;
+            const uint32_t sl = pair_k_slot(q0 + k);
 #pragma unroll
             for (int pl = 0; pl < 2; ++pl) {
               const int p = 2 * k + pl;
@@ -619,12 +618,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int i = 0; i < n && ok; ++i) {
           ok = wait_cluster(bar(C::B_PFULL + (i & 1)), (uint32_t)(i >> 1) & 1u);
           const uint32_t p_tmem = tmem + kPairPCol + 64u * (uint32_t)(i & 1);
-          const uint32_t q0 = 2u * pair_v_item(i, n);
+          const uint32_t q0 = 2u * (uint32_t)i;
 #pragma unroll
           for (int h = 0; h < 2 && ok; ++h) {
-            if (!(ok = wait_fill(q0 + h))) break;
+            if (!(ok = wait_fill(pair_v_slot(q0 + h), pair_v_phase(q0 + h)))) break;
             tc_fence_after();
-            const uint32_t sl = (q0 + h) % NSLOT;
+            const uint32_t sl = pair_v_slot(q0 + h);
 #pragma unroll
             for (int ks = 4 * h; ks < 4 * h + 4; ++ks) {
               const uint32_t off = v_offset_pair(16u * ks, 0, a.v_shift);
