@@ -93,7 +93,6 @@ struct PrefillArgs {
   int32_t q_row0;
 };
 
-
 // The work items of a balanced plan, passed by value (kernel parameter space): no device
 // allocation, and a CUDA graph that captures the launch keeps its own copy.
 struct ItemTable {
@@ -242,45 +241,6 @@ __device__ __forceinline__ uint32_t v_offset(uint32_t k, uint32_t p, int v_shift
          ((k & ((1u << v_shift) - 1u)) << 7);
 }
 
-#ifdef PA_UNIT_TIMING
-// Instrumented builds only: per CTA (blockIdx < 8192) 12 words: the global timer at entry and
-// at exit, its key-tile count with its SM in the upper half, then SM clock readings at entry,
-// after set-up, when the first S tile was seen, when the epilogue began, at exit, when the MMA
-// warp saw Q, when it saw the first K slot, when the Q tile was stored, when the first K/V copy
-// was issued, and the MMA lane's cycles waiting for K slots, V slots and P (see
-// pa_unit_timing).
-constexpr int kUnitWords = 16;
-__device__ unsigned long long g_pa_units[kUnitWords * 8192];
-__device__ __forceinline__ uint32_t smid_u32() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
-  return r;
-}
-#define PA_UNIT_ONLY(...) __VA_ARGS__
-#else
-#define PA_UNIT_ONLY(...)
-#endif
-
-#ifdef PA_TRACE
-// Instrumented builds only: cycle counters summed over all CTAs (see pa_trace_read), and an
-// event log of the first CTAs: (kind << 56 | cta << 48 | index << 32 | clock low 32 bits).
-__device__ unsigned long long g_pa_trace[16];
-constexpr int kLogCap = 1 << 16;  // 2 CTAs x 8 roles x 4096 events
-__device__ unsigned long long g_pa_log[kLogCap];
-// role: 0-2 TMA warps (or 0 the single producer), 1 MMA in the single-CTA kernel, 3 MMA,
-// 4 fill observer, 5 softmax; `n` is the role's own event counter (no atomics).
-__device__ __forceinline__ void tlog(int role, unsigned& n, int kind, int index) {
-  const unsigned long long clk = (unsigned)clock64();
-  if (blockIdx.x < 2 && n < 4096u)
-    g_pa_log[(blockIdx.x * 8 + role) * 4096 + n++] =
-        ((unsigned long long)kind << 56) | ((unsigned long long)blockIdx.x << 48) |
-        ((unsigned long long)(index & 0xFFFF) << 32) | clk;
-}
-#define PA_TRACE_ONLY(...) __VA_ARGS__
-#else
-#define PA_TRACE_ONLY(...)
-#endif
-
 // ---------------------------------------------------------------- bounded waits
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                        uint64_t timeout_ns, bool honour_abort) {
@@ -400,7 +360,6 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
     else
       mbar_arrive(addr);
   };
-  PA_TRACE_ONLY(long long tr[4] = {0, 0, 0, 0}; const long long t_begin = clock64(); unsigned tln = 0;)
   {
     const int r = threadIdx.x;  // packed Q row = tensor-memory lane
     const int64_t grow = qt * kTileRows + r;
@@ -423,8 +382,6 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       }
       fence_proxy_async_smem();
       __syncwarp();
-      PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
-                       g_pa_units[kUnitWords * blockIdx.x + 10] = clock64();)
       if (lane == 0) arrive(x.arrive_qfull);
     }
 
@@ -438,15 +395,10 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       const int sbuf = j & 1;
       const uint32_t s_col = kSCol0 + 128u * sbuf;
       const int64_t key0 = (kt0 + j) * kTileKeys;
-      PA_TRACE_ONLY(long long tw = clock64();)
       if (!warp_wait(x.bar_sfull + 8u * sbuf, (j >> 1) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
-      PA_TRACE_ONLY(const long long tc = clock64(); tr[0] += tc - tw;
-                    if (threadIdx.x == 0) tlog(5, tln, 8, j);)
-      PA_UNIT_ONLY(if (j == 0 && threadIdx.x == 0 && blockIdx.x < 8192)
-                       g_pa_units[kUnitWords * blockIdx.x + 5] = clock64();)
       tc_fence_after();
       float sv[kTileKeys];
 #pragma unroll
@@ -487,7 +439,6 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
         tc_fence_after();
         const float f = need ? ex2(m_run - m_new) : 1.0f;
         l_run *= f;
-        PA_TRACE_ONLY(tr[3] += 1;)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
@@ -535,7 +486,6 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      PA_TRACE_ONLY(if (threadIdx.x == 0) tlog(5, tln, 16, j);)
       // P lives in tensor memory: a CTA-scope release orders it (see mbar_arrive_remote_tc);
       // a tile whose V rows this thread zeroed in shared memory takes the cluster-scope one.
       if (lane == 0) {
@@ -544,28 +494,15 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
         else
           arrive(x.arrive_pfull + 8u * sbuf);
       }
-      PA_TRACE_ONLY(tr[1] += clock64() - tc; if (threadIdx.x == 0) tlog(5, tln, 9, j);)
     }
 
-    PA_TRACE_ONLY(const long long te = clock64();)
     if (ok && n >= 2)
       ok = warp_wait(x.bar_pvdone + 8u * ((n - 2) & 1), ((n - 2) >> 1) & 1, abort_flag, tmo);
     if (ok) ok = warp_wait(x.bar_pvdone + 8u * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, tmo);
-    PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
-                     g_pa_units[kUnitWords * blockIdx.x + 6] = clock64();)
     if (ok) {
       tc_fence_after();
       write_row<D>(a, x, r, valid, tok, head, m_run, l_run, t_lane);
     }
-    PA_TRACE_ONLY(tr[2] += clock64() - te;
-                  if (lane == 0) {
-                    atomicAdd(&g_pa_trace[6], (unsigned long long)tr[0]);
-                    atomicAdd(&g_pa_trace[7], (unsigned long long)tr[1]);
-                    atomicAdd(&g_pa_trace[8], (unsigned long long)tr[2]);
-                    atomicAdd(&g_pa_trace[9], (unsigned long long)tr[3]);
-                    atomicAdd(&g_pa_trace[10], (unsigned long long)(clock64() - t_begin));
-                    if (warp == 0) atomicAdd(&g_pa_trace[11], (unsigned long long)n);
-                  })
   }
 }
 
@@ -714,7 +651,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
-  PA_TRACE_ONLY(long long tr[4] = {0, 0, 0, 0}; const long long t_begin = clock64(); unsigned tln = 0;)
 
   if (warp < 4) {
     // ============================================================ softmax + epilogue
@@ -786,10 +722,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Wait until fill q's slot is free and announce its bytes; false if the wait gave up.
     auto acquire = [&](uint32_t q) -> bool {
       const uint32_t slot = q % NSLOT;
-      PA_TRACE_ONLY(const long long tw = clock64();)
       bool r_ok = q < (uint32_t)NSLOT ||
                   warp_wait(bar(C::B_EMPTY + slot), ((q / NSLOT) - 1) & 1, abort_flag, tmo);
-      PA_TRACE_ONLY(tr[0] += clock64() - tw;)
       if (r_ok && lane == 0) mbar_arrive_expect_tx(bar(C::B_FULL + slot), kPanel);
       __syncwarp();
       return r_ok;
@@ -808,7 +742,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(slot_addr(slot) + lane * prow * 128, &tm_k, bar(C::B_FULL + slot), k * 64,
                         g, row_cur);
           issued_end = q + 1;
-          PA_TRACE_ONLY(if (lane == 0) tlog(0, tln, 1, q);)
         }
       }
       if (ok && j >= 1) {  // V tile j-1: slot k holds boxes k*vbox_per_slot + lane
@@ -825,7 +758,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(slot_addr(slot) + (lane << vbytes_log), &tm_v, bar(C::B_FULL + slot), 0,
                         prow_b + (sub << a.v_shift), 0, g);
           issued_end = q + 1;
-          PA_TRACE_ONLY(if (lane == 0) tlog(0, tln, 2, q);)
         }
       }
       row_prev = row_cur;
@@ -841,10 +773,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if ((int)(q % kIssuers) == w)
         drain_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo);
     __syncwarp();
-    PA_TRACE_ONLY(if (lane == 0 && w == 0) {
-      atomicAdd(&g_pa_trace[4], (unsigned long long)tr[0]);
-      atomicAdd(&g_pa_trace[5], (unsigned long long)(clock64() - t_begin));
-    })
   } else {
     // ============================================================ MMA issuer (one lane)
     if (lane == 0) {
@@ -865,9 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t s_tmem = tmem + kSCol0 + 128u * (j & 1);
 #pragma unroll
           for (int p = 0; p < NP; ++p) {
-            PA_TRACE_ONLY(const long long tw = clock64();)
             ok = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
-            PA_TRACE_ONLY(tr[0] += clock64() - tw; tlog(1, tln, 3, j * 16 + p);)
             if (!ok) break;
             tc_fence_after();
             const uint64_t ad = q_desc + p * kSlotDesc, bd = k_desc + slot * kSlotDesc;
@@ -886,9 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (j >= 1) {
           const int i = j - 1;
-          PA_TRACE_ONLY(const long long tw = clock64();)
           ok = thread_wait(bar(C::B_PFULL + (i & 1)), (i >> 1) & 1, abort_flag, tmo);
-          PA_TRACE_ONLY(const long long tv = clock64(); tr[1] += tv - tw; tlog(1, tln, 5, i);)
           const uint32_t vslot0 = slot;  // the V tile takes slots vslot0, vslot0 + 1, ... (mod NSLOT)
 #pragma unroll
           for (int k = 0; k < NP; ++k) {
@@ -899,7 +823,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
-          PA_TRACE_ONLY(tlog(1, tln, 6, i);)
           tc_fence_after();
           const uint32_t p_tmem = tmem + kSCol0 + 128u * (i & 1) + kPColOff;
 #pragma unroll
@@ -918,16 +841,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(bar(C::B_EMPTY + vs));
           }
           umma_commit(bar(C::B_PVDONE + (i & 1)));
-          PA_TRACE_ONLY(tr[2] += clock64() - tv; tlog(1, tln, 7, i);)
         }
       }
       // Every issued MMA must finish before tensor memory is freed.
       umma_commit(bar(C::B_MMADONE));
       drain_wait(bar(C::B_MMADONE), 0, abort_flag, tmo);
-      PA_TRACE_ONLY(atomicAdd(&g_pa_trace[0], (unsigned long long)tr[0]);
-                    atomicAdd(&g_pa_trace[1], (unsigned long long)tr[1]);
-                    atomicAdd(&g_pa_trace[2], (unsigned long long)tr[2]);
-                    atomicAdd(&g_pa_trace[3], (unsigned long long)(clock64() - t_begin));)
     }
     __syncwarp();
   }
@@ -1665,44 +1583,6 @@ extern "C" int pa_device_error(int* flags, int reset) {
   if (v & kFlagTimeout) return PA_ERR_TIMEOUT;
   return PA_OK;
 }
-
-#ifdef PA_UNIT_TIMING
-extern "C" int pa_unit_timing(unsigned long long* out, int cap, int reset) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  int n = cap < kUnitWords * 8192 ? cap : kUnitWords * 8192;
-  if (cudaMemcpyFromSymbol(out, g_pa_units, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
-  if (reset) {
-    static unsigned long long z[kUnitWords * 8192];
-    cudaMemcpyToSymbol(g_pa_units, z, sizeof z);
-  }
-  return n;
-}
-#endif
-
-#ifdef PA_TRACE
-extern "C" int pa_trace_log(unsigned long long* out, int cap, int reset) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  int n = cap < kLogCap ? cap : kLogCap;
-  if (cudaMemcpyFromSymbol(out, g_pa_log, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
-  if (reset) {
-    static unsigned long long z[kLogCap];
-    cudaMemcpyToSymbol(g_pa_log, z, sizeof z);
-  }
-  return n;
-}
-// Instrumented builds only: copy (and optionally clear) the kernel's cycle counters.
-extern "C" int pa_trace_read(unsigned long long* out, int n, int reset) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
-  if (n > 16) n = 16;
-  if (cudaMemcpyFromSymbol(out, g_pa_trace, n * sizeof(unsigned long long)) != cudaSuccess)
-    return PA_ERR_CUDA;
-  if (reset) {
-    unsigned long long z[16] = {0};
-    if (cudaMemcpyToSymbol(g_pa_trace, z, sizeof z) != cudaSuccess) return PA_ERR_CUDA;
-  }
-  return PA_OK;
-}
-#endif
 
 extern "C" void pa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : 1); }
 

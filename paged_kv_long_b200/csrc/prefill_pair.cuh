@@ -152,8 +152,6 @@ __device__ __forceinline__ void softmax_pair_role(const PrefillArgs& a, const So
       ok = false;
       break;
     }
-    PA_UNIT_ONLY(if (j == 0 && threadIdx.x == 0 && blockIdx.x < 8192)
-                     g_pa_units[kUnitWords * blockIdx.x + 5] = clock64();)
     tc_fence_after();
     float sv[kTileKeys];
 #pragma unroll
@@ -262,8 +260,6 @@ __device__ __forceinline__ void softmax_pair_role(const PrefillArgs& a, const So
 
   if (ok && n >= 2) ok = wait_pv(n - 2);
   if (ok) ok = wait_pv(n - 1);
-  PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
-                   g_pa_units[kUnitWords * blockIdx.x + 6] = clock64();)
   if (ok) {
     tc_fence_after();
     write_row<D>(a, x, r, valid, tok, head, m_run, l_run, t_lane);
@@ -285,7 +281,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs
-  PA_UNIT_ONLY(const uint64_t t_entry = globaltimer_ns(); const long long c_entry = clock64();)
 
   int64_t tp, kt0, kt1;
   int g, s, slot = kSlotUniform;
@@ -372,8 +367,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
-  PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192)
-                   g_pa_units[kUnitWords * blockIdx.x + 4] = clock64();)
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = a.timeout_ns;
 
@@ -502,8 +495,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
         }
         issued = q + 1;
-        PA_UNIT_ONLY(if (q == 0 && lane == 0 && blockIdx.x < 8192)
-                         g_pa_units[kUnitWords * blockIdx.x + 11] = clock64();)
       }
     };
     // V half tile j (dims 128*rank..+127 of tile j): slot k holds keys 64k..64k+63
@@ -584,15 +575,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // half tile holds D panels 2k and 2k+1 (Q panels 2k, 2k+1). S(m) is completion m of
         // s_full and the read of S(m) arrival m of s_free.
         ok = wait_cluster(bar(C::B_QFULL), 0);
-        PA_UNIT_ONLY(if (blockIdx.x < 8192) g_pa_units[kUnitWords * blockIdx.x + 8] = clock64();)
         for (int m = 0; m < n && ok; ++m) {
           if (m >= 1) ok = wait_cluster(bar(C::B_SFREE), (uint32_t)(m - 1) & 1u);
           const uint32_t q0 = 2u * (uint32_t)m;
 #pragma unroll
           for (int k = 0; k < 2 && ok; ++k) {
             if (!(ok = wait_fill(pair_k_slot(q0 + k), pair_k_phase(q0 + k)))) break;
-            PA_UNIT_ONLY(if (m == 0 && k == 0 && blockIdx.x < 8192)
-                             g_pa_units[kUnitWords * blockIdx.x + 9] = clock64();)
             tc_fence_after();
             const uint32_t sl = pair_k_slot(q0 + k);
 #pragma unroll
@@ -650,14 +638,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  PA_UNIT_ONLY(if (threadIdx.x == 0 && blockIdx.x < 8192) {
-    unsigned long long* u = g_pa_units + kUnitWords * blockIdx.x;
-    u[0] = t_entry;
-    u[1] = globaltimer_ns();
-    u[2] = (uint64_t)n | ((uint64_t)smid_u32() << 32);
-    u[3] = (uint64_t)c_entry;
-    u[7] = (uint64_t)clock64();
-  })
   if (warp == kMmaWarp) {
     // The pair's tensor memory is freed only when both CTAs are done with it.
     if (lane == 0) mbar_arrive_remote(mapa_shared(bar(C::B_TEAR), rank ^ 1u));
