@@ -25,6 +25,11 @@ PA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Q tiles per KV head for R rows and G heads per KV head.
 PA_HD int64_t q_tiles_for(int64_t R, int G) { return ceil_div64(R * G, kTileRows); }
 
+// Decode steps whose group fits one 8-row swizzle atom at head dim 128 or 256 run the kernel
+// with swapped operands, two CTAs per SM (pa_decode_plan sizes its splits for those slots).
+constexpr int kDecCtasPerSm = 2;
+PA_HD bool decode_swapped(int D, int G) { return G <= 8 && (D == 128 || D == 256); }
+
 // Last token (chunk-relative, inclusive) held by Q tile qt.
 PA_HD int64_t tile_last_token(int64_t qt, int64_t R, int G) {
   const int64_t t = (qt * kTileRows + kTileRows - 1) / G;

@@ -211,12 +211,20 @@ __device__ __noinline__ int seq_of_class_rank(const int32_t* lens, int B, int r,
 // loaded as one TMA box per (page, panel). A V tile is a run of TMA boxes of v_rows keys x
 // all NP panels (each box panel-major, the MN-major B operand of P V); a box never straddles
 // two slots. Fill number q is issued by TMA warp q % kIssuers.
-template <int D>
+// SQ (small Q): every Q tile of the launch holds at most 8 packed rows (decode: one token of
+// G <= 8 heads). Q then takes one 8-row swizzle atom per panel (1 KB, not 16 KB) and the
+// A operand of Q K^T repeats that atom over the 128 rows of the MMA (descriptor stride 0):
+// rows 8..127 of S are copies of rows 0..7, which belong to no output. The freed 60 KB
+// deepen the ring to 13 slots, so the copies run further ahead of a unit that is bound by
+// its K/V reads.
+template <int D, bool SQ = false>
 struct Cfg {
   static constexpr int NP = D / 64;                  // 64-element panels per K/V/Q row
-  static constexpr int NSLOT = (D == 256) ? 10 : 12; // ring of 16 KB slots
+  static constexpr int NSLOT = SQ ? 13 : (D == 256) ? 10 : 12;  // ring of 16 KB slots
+  static constexpr int Q_PANEL = SQ ? 1024 : kPanel; // bytes of one Q panel
+  static constexpr int Q_SBO = SQ ? 0 : 1024;        // Q descriptor: bytes between 8-row atoms
   static constexpr int Q_OFF = 0;
-  static constexpr int RING_OFF = Q_OFF + NP * kPanel;
+  static constexpr int RING_OFF = Q_OFF + NP * Q_PANEL;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * kPanel;
   // barriers: full[NSLOT], empty[NSLOT], q_full, s_full[2], p_full[2], pv_done[2], mma_done
   static constexpr int B_FULL = 0, B_EMPTY = NSLOT, B_QFULL = 2 * NSLOT, B_SFULL = 2 * NSLOT + 1,
@@ -344,7 +352,7 @@ __device__ __forceinline__ void write_row(const PrefillArgs& a, const SoftmaxCtx
   if (valid && ws_row >= 0) a.ws_lse[ws_row] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
 }
 
-template <int D, bool PAGED, bool BF16, class VTail>
+template <int D, bool PAGED, bool BF16, bool SQ, class VTail>
 __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const SoftmaxCtx& x,
                                              VTail&& v_tail) {
   constexpr int NP = D / 64;
@@ -368,16 +376,20 @@ __device__ __forceinline__ void softmax_role(const PrefillArgs& a, const Softmax
     const int head = g * a.G + (int)(grow % a.G);
     if (!a.q_tma) {
       // Q tile -> shared memory as K-major rows of 64-element panels, 128-byte swizzle (when
-      // the tensor copy cannot: it loads whole tokens, so it needs G to divide 128).
+      // the tensor copy cannot: it loads whole tokens, so it needs G to divide 128). Small Q:
+      // rows 0..7 only, one 1 KB atom per panel.
+      constexpr uint32_t kQPanel = SQ ? 1024u : (uint32_t)kPanel;
       const uint4* src =
           reinterpret_cast<const uint4*>(a.q + (valid ? (tok * a.Hq + head) * (int64_t)D : 0));
+      if (!SQ || r < 8) {
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
+        for (int p = 0; p < NP; ++p) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = valid ? __ldg(src + p * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
-          st_shared_v4(sb + x.q_off + p * kPanel + r * 128 + ((c ^ (r & 7)) << 4), v.x, v.y, v.z,
-                       v.w);
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = valid ? __ldg(src + p * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+            st_shared_v4(sb + x.q_off + p * kQPanel + r * 128 + ((c ^ (r & 7)) << 4), v.x, v.y,
+                         v.z, v.w);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -529,13 +541,162 @@ __device__ __forceinline__ int32_t tile_page_row(const PrefillArgs& a, int64_t k
   return row;
 }
 
+// Device-length decode, block blockIdx.x: unit (sequence of rank blockIdx.x / (Hkv·S), KV head
+// g, split s) over its keys 0 .. len-1 (the new token's own included, all visible). Points a at
+// the sequence (Q, output and workspace rows, page-table row, lengths) and gives the unit's KV
+// tiles [kt0, kt1). A length outside 0 .. the table row's keys is reported like a bad page
+// entry and clamped. Every thread of the block takes part (block barriers in the ranking);
+// `scratch`: shared memory that no copy writes yet (see seq_of_rank).
+template <int D>
+__device__ __forceinline__ void decode_unit(PrefillArgs& a, int32_t* scratch, int* g, int* s,
+                                            int64_t* kt0, int64_t* kt1) {
+  const int64_t per_seq = (int64_t)a.Hkv * a.splits;
+  const int64_t rem = blockIdx.x % per_seq;
+  int64_t b = blockIdx.x / per_seq;
+  b = a.batch <= kRankedSeqsMax ? seq_of_rank(a.seq_lens, a.batch, (int)b, scratch)
+                                : seq_of_class_rank(a.seq_lens, a.batch, (int)b, scratch);
+  *g = (int)(rem / a.splits);
+  *s = (int)(rem % a.splits);
+  int64_t len = __ldg(a.seq_lens + b);
+  const int64_t cap = (int64_t)a.table_stride * a.page_rows;  // keys the table row can map
+  if (len < 0 || len > cap) {
+    if (threadIdx.x == 0 && *g == 0 && *s == 0) atomicOr(&g_pa_error_flags, kFlagPage);
+    len = len < 0 ? 0 : cap;
+  }
+  a.q += b * a.Hq * D;
+  a.out += b * a.Hq * D;
+  if (a.ws_o) {
+    a.ws_o += b * a.Hq * D;
+    a.ws_lse += b * a.Hq;
+  }
+  a.page_table += b * a.table_stride;
+  a.hist_len = len > 0 ? len - 1 : 0;
+  a.total_keys = len;
+  a.table_len = (len + a.page_rows - 1) / a.page_rows;
+  a.R = len > 0 ? 1 : 0;
+  split_range((len + kTileKeys - 1) / kTileKeys, *s, a.splits, kt0, kt1);
+}
+
+// A unit without KV tiles (a split past its tile's keys, or a decode sequence with no key):
+// zeros for the output (one split) or an empty partial (zeros, LSE -inf), by threads < 128.
+template <int D>
+__device__ __forceinline__ void empty_unit(const PrefillArgs& a, int64_t qt, int g, int s) {
+  if (threadIdx.x >= kTileRows) return;
+  const int64_t grow = qt * kTileRows + threadIdx.x;
+  const int64_t tok = grow / a.G;
+  if (tok >= (a.batch > 0 ? 1 : a.R)) return;
+  const int head = g * a.G + (int)(grow % a.G);
+  if (a.splits == 1) {
+    float4* d4 = reinterpret_cast<float4*>(a.out + (tok * a.Hq + head) * D);
+    for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    const int64_t row = (int64_t)s * a.ws_split_rows + tok * a.Hq + head;
+    float4* d4 = reinterpret_cast<float4*>(a.ws_o + row * D);
+    for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    a.ws_lse[row] = -INFINITY;
+  }
+}
+
+// The copy warps of the single-CTA kernels (warp w of kIssuers): fill the ring of NSLOT 16 KB
+// slots at `ring` in the order K0, K1, V0, K2, V1, ..., V_{n-1} (see Cfg) for the n KV tiles
+// kt0 .. kt0 + n - 1 of KV head g, fill number q by warp q % kIssuers. full[i] / empty[i] are the slots'
+// barriers (8 bytes apart). pre_row0 / pre_row1: lane i's page row of tiles 0 / 1 (read
+// before the set-up). Every copy has landed when this returns.
+template <int NP, int NSLOT, int PANEL_LOG, bool PAGED>
+__device__ __forceinline__ void kv_copy_role(const PrefillArgs& a, const CUtensorMap* tm_k,
+                                             const CUtensorMap* tm_v, int g, int64_t kt0, int n,
+                                             int w, uint32_t ring, uint32_t bar_full, uint32_t bar_empty,
+                                             int32_t pre_row0, int32_t pre_row1,
+                                             volatile int* abort_flag, uint64_t tmo) {
+  const int lane = threadIdx.x & 31;
+  auto slot_addr = [&](uint32_t slot) -> uint32_t { return ring + slot * kPanel; };
+  auto full = [&](uint32_t slot) -> uint32_t { return bar_full + 8u * slot; };
+  const int ppt = a.pages_per_tile;   // pages per KV tile (1 when contiguous)
+  const int prow = a.page_rows;       // key rows per page (kTileKeys when contiguous)
+  const int vsub = prow >> a.v_shift; // V boxes per page
+  const int vbytes_log = a.v_shift + PANEL_LOG;   // log2 of a V box's bytes
+  const int vbox_per_slot = 1 << (14 - vbytes_log);
+  bool ok = true;
+  // Lane i < ppt holds the key-row coordinate of page i of a tile (read one tile ahead).
+  auto fetch = [&](int jt) -> int32_t {
+    int32_t row = a.oob_row;
+    if constexpr (PAGED) {
+      const int64_t lp = (kt0 + jt) * ppt + lane;
+      if (jt < n && lane < ppt && lp < a.table_len) {
+        const int32_t e = __ldg(a.page_table + lp);
+        if (e >= 0 && e < a.num_pages)
+          row = e << a.page_shift;
+        else if (w == 0)
+          atomicOr(&g_pa_error_flags, kFlagPage);
+      }
+    } else {
+      row = (int32_t)((kt0 + jt) * kTileKeys);
+    }
+    return row;
+  };
+  // Wait until fill q's slot is free and announce its bytes; false if the wait gave up.
+  auto acquire = [&](uint32_t q) -> bool {
+    const uint32_t slot = q % NSLOT;
+    bool r_ok = q < (uint32_t)NSLOT ||
+                warp_wait(bar_empty + 8u * slot, ((q / NSLOT) - 1) & 1, abort_flag, tmo);
+    if (r_ok && lane == 0) mbar_arrive_expect_tx(full(slot), kPanel);
+    __syncwarp();
+    return r_ok;
+  };
+  int32_t row_prev = a.oob_row, row_cur = pre_row0, row_next = pre_row1;
+  uint32_t issued_end = 0;  // one past the last fill number this warp issued
+  for (int j = 0; j <= n && ok; ++j) {
+    if (j < n) {  // K tile j: panel k in fill q, one box per page (lane i: page i)
+      const uint32_t item = j == 0 ? 0u : 2u * j - 1u;
+      for (int k = 0; k < NP && ok; ++k) {
+        const uint32_t q = item * NP + k;
+        if ((int)(q % kIssuers) != w) continue;
+        if (!(ok = acquire(q))) break;
+        const uint32_t slot = q % NSLOT;
+        if (lane < ppt)
+          tma_load_3d(slot_addr(slot) + lane * prow * 128, tm_k, full(slot), k * 64, g,
+                      row_cur);
+        issued_end = q + 1;
+      }
+    }
+    if (ok && j >= 1) {  // V tile j-1: slot k holds boxes k*vbox_per_slot + lane
+      const uint32_t item = v_item(j - 1, n);
+      for (int k = 0; k < NP && ok; ++k) {
+        const uint32_t q = item * NP + k;
+        if ((int)(q % kIssuers) != w) continue;
+        if (!(ok = acquire(q))) break;
+        const uint32_t slot = q % NSLOT;
+        const int b = k * vbox_per_slot + lane;        // box index inside the V tile
+        const int pg = b / vsub, sub = b - pg * vsub;  // its page and place in the page
+        const int32_t prow_b = __shfl_sync(0xffffffffu, row_prev, pg & 31);
+        if (lane < vbox_per_slot)
+          tma_load_4d(slot_addr(slot) + (lane << vbytes_log), tm_v, full(slot), 0,
+                      prow_b + (sub << a.v_shift), 0, g);
+        issued_end = q + 1;
+      }
+    }
+    row_prev = row_cur;
+    row_cur = row_next;
+    row_next = fetch(j + 2);
+  }
+  // Every copy must land before the CTA may exit. Only the last fill of each slot is still
+  // waitable by parity (an earlier one may be two phases back), so each warp waits for its
+  // own fills among the last NSLOT of the whole sequence; fills it never issued (after an
+  // abort) are skipped.
+  const uint32_t all_fills = 2u * n * NP;
+  for (uint32_t q = all_fills > (uint32_t)NSLOT ? all_fills - NSLOT : 0; q < issued_end; ++q)
+    if ((int)(q % kIssuers) == w)
+      drain_wait(full(q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo);
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------- prefill kernel
-template <int D, bool PAGED, bool BF16>
+template <int D, bool PAGED, bool BF16, bool SQ>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const PrefillArgs a_in, const __grid_constant__ ItemTable items) {
   PrefillArgs a = a_in;  // rebased on one sequence in batched plans and decode
-  using C = Cfg<D>;
+  using C = Cfg<D, SQ>;
   constexpr int NP = C::NP, NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
@@ -554,34 +715,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     kt1 = it.kt1;
     slot = it.slot;
   } else if (a.batch > 0) {
-    // one new token of sequence b: keys 0 .. len-1 (its own included), all visible
-    const int64_t per_seq = (int64_t)a.Hkv * a.splits;
-    const int64_t rem = blockIdx.x % per_seq;
-    int64_t b = blockIdx.x / per_seq;
-    int32_t* scratch = reinterpret_cast<int32_t*>(smem + C::RING_OFF);
-    b = a.batch <= kRankedSeqsMax ? seq_of_rank(a.seq_lens, a.batch, (int)b, scratch)
-                                  : seq_of_class_rank(a.seq_lens, a.batch, (int)b, scratch);
-    g = (int)(rem / a.splits);
-    s = (int)(rem % a.splits);
+    decode_unit<D>(a, reinterpret_cast<int32_t*>(smem + C::RING_OFF), &g, &s, &kt0, &kt1);
     qt = 0;
-    int64_t len = __ldg(a.seq_lens + b);
-    const int64_t cap = (int64_t)a.table_stride * a.page_rows;  // keys the table row can map
-    if (len < 0 || len > cap) {  // reported like a bad page entry; the length is clamped
-      if (threadIdx.x == 0 && g == 0 && s == 0) atomicOr(&g_pa_error_flags, kFlagPage);
-      len = len < 0 ? 0 : cap;
-    }
-    a.q += b * a.Hq * D;
-    a.out += b * a.Hq * D;
-    if (a.ws_o) {
-      a.ws_o += b * a.Hq * D;
-      a.ws_lse += b * a.Hq;
-    }
-    a.page_table += b * a.table_stride;
-    a.hist_len = len > 0 ? len - 1 : 0;
-    a.total_keys = len;
-    a.table_len = (len + a.page_rows - 1) / a.page_rows;
-    a.R = len > 0 ? 1 : 0;
-    split_range((len + kTileKeys - 1) / kTileKeys, s, a.splits, &kt0, &kt1);
   } else {
     unit_coords(blockIdx.x, a.q_tiles, a.Hkv, a.splits, &qt, &g, &s);
     split_range(tile_kv_tiles(qt, a.R, a.G, a.hist_len), s, a.splits, &kt0, &kt1);
@@ -589,22 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = (int)(kt1 - kt0);
 
   if (n == 0) {  // a split past this tile's keys (only when S > KV tiles): empty partial
-    if (threadIdx.x < kTileRows) {
-      const int64_t grow = qt * kTileRows + threadIdx.x;
-      const int64_t tok = grow / a.G;
-      if (tok < (a.batch > 0 ? 1 : a.R)) {
-        const int head = g * a.G + (int)(grow % a.G);
-        if (a.splits == 1) {  // decode of a sequence with no key: zeros
-          float4* d4 = reinterpret_cast<float4*>(a.out + (tok * a.Hq + head) * D);
-          for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          const int64_t row = (int64_t)s * a.ws_split_rows + tok * a.Hq + head;
-          float4* d4 = reinterpret_cast<float4*>(a.ws_o + row * D);
-          for (int i = 0; i < D / 4; ++i) d4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          a.ws_lse[row] = -INFINITY;
-        }
-      }
-    }
+    empty_unit<D>(a, qt, g, s);
     return;
   }
 
@@ -692,87 +812,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       return true;
     };
-    softmax_role<D, PAGED, BF16>(a, sc, v_tail);
+    softmax_role<D, PAGED, BF16, SQ>(a, sc, v_tail);
   } else if (warp > kMmaWarp) {
     // ============================================================ TMA issuers (three warps)
-    const int w = warp - kMmaWarp - 1;  // this warp issues fill numbers q with q % kIssuers == w
-    const int ppt = a.pages_per_tile;   // pages per KV tile (1 when contiguous)
-    const int prow = a.page_rows;       // key rows per page (kTileKeys when contiguous)
-    const int vsub = prow >> a.v_shift; // V boxes per page
-    const int vbytes_log = a.v_shift + C::PANEL_LOG;   // log2 of a V box's bytes
-    const int vbox_per_slot = 1 << (14 - vbytes_log);
-    bool ok = true;
-    // Lane i < ppt holds the key-row coordinate of page i of a tile (read one tile ahead).
-    auto fetch = [&](int jt) -> int32_t {
-      int32_t row = a.oob_row;
-      if constexpr (PAGED) {
-        const int64_t lp = (kt0 + jt) * ppt + lane;
-        if (jt < n && lane < ppt && lp < a.table_len) {
-          const int32_t e = __ldg(a.page_table + lp);
-          if (e >= 0 && e < a.num_pages)
-            row = e << a.page_shift;
-          else if (w == 0)
-            atomicOr(&g_pa_error_flags, kFlagPage);
-        }
-      } else {
-        row = (int32_t)((kt0 + jt) * kTileKeys);
-      }
-      return row;
-    };
-    // Wait until fill q's slot is free and announce its bytes; false if the wait gave up.
-    auto acquire = [&](uint32_t q) -> bool {
-      const uint32_t slot = q % NSLOT;
-      bool r_ok = q < (uint32_t)NSLOT ||
-                  warp_wait(bar(C::B_EMPTY + slot), ((q / NSLOT) - 1) & 1, abort_flag, tmo);
-      if (r_ok && lane == 0) mbar_arrive_expect_tx(bar(C::B_FULL + slot), kPanel);
-      __syncwarp();
-      return r_ok;
-    };
-    int32_t row_prev = a.oob_row, row_cur = pre_row0, row_next = pre_row1;
-    uint32_t issued_end = 0;  // one past the last fill number this warp issued
-    for (int j = 0; j <= n && ok; ++j) {
-      if (j < n) {  // K tile j: panel k in fill q, one box per page (lane i: page i)
-        const uint32_t item = j == 0 ? 0u : 2u * j - 1u;
-        for (int k = 0; k < NP && ok; ++k) {
-          const uint32_t q = item * NP + k;
-          if ((int)(q % kIssuers) != w) continue;
-          if (!(ok = acquire(q))) break;
-          const uint32_t slot = q % NSLOT;
-          if (lane < ppt)
-            tma_load_3d(slot_addr(slot) + lane * prow * 128, &tm_k, bar(C::B_FULL + slot), k * 64,
-                        g, row_cur);
-          issued_end = q + 1;
-        }
-      }
-      if (ok && j >= 1) {  // V tile j-1: slot k holds boxes k*vbox_per_slot + lane
-        const uint32_t item = v_item(j - 1, n);
-        for (int k = 0; k < NP && ok; ++k) {
-          const uint32_t q = item * NP + k;
-          if ((int)(q % kIssuers) != w) continue;
-          if (!(ok = acquire(q))) break;
-          const uint32_t slot = q % NSLOT;
-          const int b = k * vbox_per_slot + lane;        // box index inside the V tile
-          const int pg = b / vsub, sub = b - pg * vsub;  // its page and place in the page
-          const int32_t prow_b = __shfl_sync(0xffffffffu, row_prev, pg & 31);
-          if (lane < vbox_per_slot)
-            tma_load_4d(slot_addr(slot) + (lane << vbytes_log), &tm_v, bar(C::B_FULL + slot), 0,
-                        prow_b + (sub << a.v_shift), 0, g);
-          issued_end = q + 1;
-        }
-      }
-      row_prev = row_cur;
-      row_cur = row_next;
-      row_next = fetch(j + 2);
-    }
-    // Every copy must land before the CTA may exit. Only the last fill of each slot is still
-    // waitable by parity (an earlier one may be two phases back), so each warp waits for its
-    // own fills among the last NSLOT of the whole sequence; fills it never issued (after an
-    // abort) are skipped.
-    const uint32_t all_fills = 2u * n * NP;
-    for (uint32_t q = all_fills > (uint32_t)NSLOT ? all_fills - NSLOT : 0; q < issued_end; ++q)
-      if ((int)(q % kIssuers) == w)
-        drain_wait(bar(C::B_FULL + q % NSLOT), (q / NSLOT) & 1, abort_flag, tmo);
-    __syncwarp();
+    kv_copy_role<NP, NSLOT, C::PANEL_LOG, PAGED>(a, &tm_k, &tm_v, g, kt0, n,
+                                                 warp - kMmaWarp - 1, sb + C::RING_OFF,
+                                                 bar(C::B_FULL), bar(C::B_EMPTY), pre_row0,
+                                                 pre_row1, abort_flag, tmo);
   } else {
     // ============================================================ MMA issuer (one lane)
     if (lane == 0) {
@@ -780,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = umma_idesc_f16(128, D, BF16, true);
       constexpr uint32_t kSlotDesc = kPanel >> 4;  // descriptor units per slot
       // Descriptor templates; the start address field takes plain additions of (bytes >> 4).
-      const uint64_t q_desc = smem_desc_sw128(sb + C::Q_OFF, 16, 1024);
+      const uint64_t q_desc = smem_desc_sw128(sb + C::Q_OFF, 16, C::Q_SBO);
       const uint64_t k_desc = smem_desc_sw128(sb + C::RING_OFF, 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(sb + C::RING_OFF, (uint32_t)a.v_rows * 128u, 1024);
       uint32_t slot = 0, round = 0;
@@ -796,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = thread_wait(bar(C::B_FULL + slot), round & 1, abort_flag, tmo);
             if (!ok) break;
             tc_fence_after();
-            const uint64_t ad = q_desc + p * kSlotDesc, bd = k_desc + slot * kSlotDesc;
+            const uint64_t ad = q_desc + p * (C::Q_PANEL >> 4), bd = k_desc + slot * kSlotDesc;
             umma_ss(s_tmem, ad, bd, idesc_qk, p != 0 ? 1u : 0u);
             umma_ss(s_tmem, ad + 2, bd + 2, idesc_qk, 1u);
             umma_ss(s_tmem, ad + 4, bd + 4, idesc_qk, 1u);
@@ -859,6 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 #include "prefill_pair.cuh"
+#include "decode_kernel.cuh"
 #include "kv_append.cuh"
 
 // ---------------------------------------------------------------- combine kernels
@@ -1067,10 +1114,10 @@ bool make_q_map(CUtensorMap* map, const void* base, bool bf16, int D, int G, int
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool PAGED, bool BF16>
+template <int D, bool PAGED, bool BF16, bool SQ = false>
 cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
                            const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
-  auto kern = prefill_kernel<D, PAGED, BF16>;
+  auto kern = prefill_kernel<D, PAGED, BF16, SQ>;
   static std::atomic<uint64_t> configured{0};  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1078,11 +1125,11 @@ cudaError_t launch_prefill(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg<D>::LAUNCH_SMEM);
+                             Cfg<D, SQ>::LAUNCH_SMEM);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  kern<<<(unsigned)grid, kThreads, Cfg<D>::LAUNCH_SMEM, st>>>(tk, tv, a, it);
+  kern<<<(unsigned)grid, kThreads, Cfg<D, SQ>::LAUNCH_SMEM, st>>>(tk, tv, a, it);
   return cudaGetLastError();
 }
 
@@ -1127,6 +1174,50 @@ cudaError_t launch_d(bool paged, bool bf16, int64_t grid, cudaStream_t st, const
                 : launch_prefill<D, true, false>(grid, st, tk, tv, a, it);
   return bf16 ? launch_prefill<D, false, true>(grid, st, tk, tv, a, it)
               : launch_prefill<D, false, false>(grid, st, tk, tv, a, it);
+}
+
+template <int D, bool BF16>
+cudaError_t launch_decode(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const PrefillArgs& a) {
+  auto kern = decode_kernel<D, BF16>;
+  static std::atomic<uint64_t> configured{0};  // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecCfg<D>::LAUNCH_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  kern<<<(unsigned)grid, kThreads, DecCfg<D>::LAUNCH_SMEM, st>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+
+// Paged single-CTA launches of decode and batches (sq: every Q tile holds <= 8 packed rows).
+cudaError_t launch_paged_single(int D, bool bf16, bool sq, int64_t grid, cudaStream_t st,
+                                const CUtensorMap& tk, const CUtensorMap& tv,
+                                const PrefillArgs& a, const ItemTable& it) {
+  if (sq) {
+    switch (D) {
+      case 64: return bf16 ? launch_prefill<64, true, true, true>(grid, st, tk, tv, a, it)
+                           : launch_prefill<64, true, false, true>(grid, st, tk, tv, a, it);
+      case 128: return bf16 ? launch_prefill<128, true, true, true>(grid, st, tk, tv, a, it)
+                            : launch_prefill<128, true, false, true>(grid, st, tk, tv, a, it);
+      default: return bf16 ? launch_prefill<256, true, true, true>(grid, st, tk, tv, a, it)
+                           : launch_prefill<256, true, false, true>(grid, st, tk, tv, a, it);
+    }
+  }
+  switch (D) {
+    case 64: return launch_d<64>(true, bf16, grid, st, tk, tv, a, it);
+    case 128: return launch_d<128>(true, bf16, grid, st, tk, tv, a, it);
+    default: return bf16 ? launch_prefill<256, true, true>(grid, st, tk, tv, a, it)
+                         : launch_prefill<256, true, false>(grid, st, tk, tv, a, it);
+  }
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -1310,14 +1401,13 @@ extern "C" int pa_decode(const pa_plan_t* plan, const void* q, const void* k_poo
   const int64_t grid = plan->units;
   if (grid >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   cudaError_t e;
-  switch (D) {
-    case 64: e = bf16 ? launch_prefill<64, true, true>(grid, st, tk, tv, a, table)
-                      : launch_prefill<64, true, false>(grid, st, tk, tv, a, table); break;
-    case 128: e = bf16 ? launch_prefill<128, true, true>(grid, st, tk, tv, a, table)
-                       : launch_prefill<128, true, false>(grid, st, tk, tv, a, table); break;
-    default: e = bf16 ? launch_prefill<256, true, true>(grid, st, tk, tv, a, table)
-                      : launch_prefill<256, true, false>(grid, st, tk, tv, a, table); break;
-  }
+  if (decode_swapped(D, plan->group))
+    e = D == 128 ? (bf16 ? launch_decode<128, true>(grid, st, tk, tv, a)
+                         : launch_decode<128, false>(grid, st, tk, tv, a))
+                 : (bf16 ? launch_decode<256, true>(grid, st, tk, tv, a)
+                         : launch_decode<256, false>(grid, st, tk, tv, a));
+  else
+    e = launch_paged_single(D, bf16, plan->group <= 8, grid, st, tk, tv, a, table);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -1451,19 +1541,15 @@ extern "C" int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens,
   for (size_t i = 0; i < bt.seq.size(); ++i) table.seq[i] = bt.seq[i];
   const int64_t grid = plan->units * per;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int max_rows = 0;  // small Q when no sequence's Q tile holds more than 8 packed rows
+  for (const PaSeq& sq : bt.seq) max_rows = std::max(max_rows, (int)sq.rows);
+  const bool small_q = (int64_t)max_rows * plan->group <= 8;
   cudaError_t e;
-  switch (D) {
-    case 64: e = launch_d<64>(true, bf16, grid, cs, tk, tv, a, table); break;
-    case 128: e = launch_d<128>(true, bf16, grid, cs, tk, tv, a, table); break;
-    default:
-      if (per == 2)
-        e = bf16 ? launch_pair<true, true>(grid, cs, tk, tv, tq, a, table)
-                 : launch_pair<true, false>(grid, cs, tk, tv, tq, a, table);
-      else
-        e = bf16 ? launch_prefill<256, true, true>(grid, cs, tk, tv, a, table)
-                 : launch_prefill<256, true, false>(grid, cs, tk, tv, a, table);
-      break;
-  }
+  if (per == 2)
+    e = bf16 ? launch_pair<true, true>(grid, cs, tk, tv, tq, a, table)
+             : launch_pair<true, false>(grid, cs, tk, tv, tq, a, table);
+  else
+    e = launch_paged_single(D, bf16, small_q, grid, cs, tk, tv, a, table);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

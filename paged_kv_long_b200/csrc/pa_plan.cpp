@@ -447,8 +447,10 @@ extern "C" int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int he
   if (max_seq_len + pa::kTileKeys >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   const int64_t max_tiles = pa::ceil_div64(max_seq_len, pa::kTileKeys);
   int S = splits_override;
-  if (S == 0) {  // about two units per SM
-    const int64_t want = pa::ceil_div64(2LL * num_sms, (int64_t)batch * n_kv_heads);
+  if (S == 0) {  // about two units per CTA slot (two slots per SM for the swapped kernel)
+    const int64_t slots =
+        (int64_t)num_sms * (pa::decode_swapped(head_dim, G) ? pa::kDecCtasPerSm : 1);
+    const int64_t want = pa::ceil_div64(2 * slots, (int64_t)batch * n_kv_heads);
     S = (int)std::max<int64_t>(1, std::min<int64_t>({want, (int64_t)PA_MAX_SPLITS, max_tiles}));
   }
   if ((int64_t)batch * n_kv_heads * S >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;

@@ -114,7 +114,8 @@ def test_decode_plan_fields_and_workspace():
     p = bd.decode_plan(16, 2, 256, 16, batch=8, max_seq_len=32768, dtype="f16", num_sms=148)
     assert p.batch == 8 and p.chunk_rows == 8 and p.q_tiles == 1 and p.ctas_per_unit == 1
     S = p.splits
-    assert S == min(32, math.ceil(2 * 148 / (8 * 2)))
+    # G = 8 at head dim 256: the swapped-operand kernel, two CTA slots per SM, two units each
+    assert S == min(32, math.ceil(2 * 2 * 148 / (8 * 2)))
     assert p.units == 8 * 2 * S
     assert p.ws_bytes == S * 8 * 16 * (256 + 1) * 4
     assert abs(p.scale - 1 / 16) < 1e-7
@@ -124,8 +125,13 @@ def test_decode_plan_splits_bounded_by_tiles_and_override():
     bd = _binding()
     p = bd.decode_plan(8, 1, 128, 16, batch=1, max_seq_len=300, dtype="bf16", num_sms=148)
     assert p.splits == 3                     # three 128-key tiles
+    # the batch alone gives two units per CTA slot (2 x 148 slots of the swapped kernel)
+    p = bd.decode_plan(8, 1, 128, 16, batch=600, max_seq_len=1 << 20, dtype="bf16", num_sms=148)
+    assert p.splits == 1 and p.ws_bytes == 0
     p = bd.decode_plan(8, 1, 128, 16, batch=512, max_seq_len=1 << 20, dtype="bf16", num_sms=148)
-    assert p.splits == 1 and p.ws_bytes == 0  # the batch alone fills the SMs
+    assert p.splits == 2
+    p = bd.decode_plan(16, 1, 128, 16, batch=512, max_seq_len=1 << 20, dtype="bf16", num_sms=148)
+    assert p.splits == 1                      # G = 16: one CTA slot per SM
     p = bd.decode_plan(8, 1, 128, 16, batch=2, max_seq_len=4096, dtype="bf16", splits=5,
                        num_sms=148)
     assert p.splits == 5 and p.units == 2 * 1 * 5
@@ -172,6 +178,11 @@ CASES = [
     ("d64_g16", [700, 64, 1500], 32, 2, 64, 128, "f16", 0),
     ("d64_g1", [33, 800], 4, 4, 64, 16, "bf16", 4),
     ("d64_24_splits", [3000, 5, 130], 8, 1, 64, 16, "f16", 24),
+    # G > 8 at head dim 256: the single-CTA kernel with a whole Q tile (not the swapped one)
+    ("d256_g16_unswapped", [2000, 129, 5], 32, 2, 256, 16, "bf16", 0),
+    # the swapped kernel with V boxes of 32 keys (D 256) and 64 keys (D 128)
+    ("d256_ps128", [5000, 128, 1, 257], 8, 1, 256, 128, "f16", 0),
+    ("d128_ps128_g8", [4000, 700, 0, 129], 16, 2, 128, 128, "bf16", 0),
 ]
 
 
@@ -232,17 +243,20 @@ def test_gpu_decode_long_batch_sampled():
 
 @pytest.mark.gpu
 @pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
-@pytest.mark.parametrize("B,max_len,Hkv", [(255, 400, 2), (256, 400, 2), (257, 400, 2),
-                                            (700, 400, 2), (600, 6000, 1)])
-def test_gpu_decode_longest_first_dispatch_edges(B, max_len, Hkv):
+@pytest.mark.parametrize("B,max_len,Hkv,D", [(255, 400, 2, 64), (256, 400, 2, 64),
+                                              (257, 400, 2, 64), (700, 400, 2, 64),
+                                              (600, 6000, 1, 64), (256, 1500, 2, 256),
+                                              (300, 1500, 1, 128)])
+def test_gpu_decode_longest_first_dispatch_edges(B, max_len, Hkv, D):
     """Blocks go to sequences longest first (ties by index) up to 256 sequences, and by length
     class (floor(log2(KV tiles)), sequence order within a class) beyond: both sides of that
-    edge, with runs of equal lengths and empty sequences, every output against the oracle."""
+    edge, with runs of equal lengths and empty sequences, every output against the oracle
+    (head dim 64 on the single-CTA kernel, 128 and 256 on the swapped one)."""
     rng = np.random.default_rng(800 + B)
     lens = rng.integers(0, max_len, size=B)
     lens[::7] = 129          # a run of ties across the batch
     lens[3::11] = 0
-    db = decode_batch(801 + B, lens, 4 * Hkv, Hkv, 64, 16, "f16")
+    db = decode_batch(801 + B, lens, 4 * Hkv, Hkv, D, 16, "f16")
     p, got = run_decode(db, splits=3)
     assert _binding().device_error(reset=True)[0] == 0
     empty = db.seq_lens == 0
@@ -299,14 +313,15 @@ def test_gpu_decode_graph_replay_follows_device_lengths():
 
 @pytest.mark.gpu
 @pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")
-def test_gpu_decode_length_past_table_is_reported():
+@pytest.mark.parametrize("D", [64, 256])
+def test_gpu_decode_length_past_table_is_reported(D):
     import torch
     bd = _binding()
     bd.device_error(reset=True)
-    db = decode_batch(79, [40, 20], 4, 2, 64, 16, "f16")
+    db = decode_batch(79, [40, 20], 4, 2, D, 16, "f16")
     lens = db.seq_lens.copy()
     lens[1] = db.block_table.shape[1] * 16 + 1  # more keys than the table row maps
-    p = bd.decode_plan(4, 2, 64, 16, 2, 64, "f16")
+    p = bd.decode_plan(4, 2, D, 16, 2, 64, "f16")
     bd.decode(p, _dev(db.q, "f16"), _dev(db.k_pool, "f16"), _dev(db.v_pool, "f16"),
               torch.from_numpy(db.block_table).cuda(), torch.from_numpy(lens).cuda())
     st, flags = bd.device_error(reset=True)
