@@ -79,6 +79,7 @@ struct PrefillArgs {
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
   int32_t q_tma;           // 1: the Q tile arrives by tensor copy (CTA-pair kernel, G | 128)
+  int32_t k_atoms;         // 1: a K box is 8 keys x all 4 panels (CTA-pair kernel, pages of 16)
   int64_t ws_split_rows;   // workspace rows of one split: R * Hq (decode: batch * Hq)
   // Batched decode (batch > 0, single-CTA kernel): unit u is (sequence u / (Hkv*S), KV head,
   // split); sequence b has seq_lens[b] keys, its page-table row at page_table + b * table_stride,
@@ -1275,7 +1276,11 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   const int k_rows = per == 2 ? std::min(page_rows, 64) : page_rows;
   const int v_rows = per == 2 ? std::min(page_rows, 64) : std::min(page_rows, 128 / (D / 64));
   const int v_panels = per == 2 ? 2 : D / 64;
-  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows) ||
+  // CTA pair, pages of 16 keys: K in boxes of 8 keys x all of D (one swizzle atom per panel),
+  // 8 boxes per half tile instead of 16 one-panel boxes of a page each
+  const bool k_atoms = per == 2 && page_rows == 16;
+  if (!(k_atoms ? make_v_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, 8, D / 64)
+                : make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows)) ||
       !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, v_panels))
     return PA_ERR_CUDA;
   // CTA pair: Q by tensor copy when a packed 128-row tile is whole tokens
@@ -1319,6 +1324,7 @@ extern "C" int pa_prefill(const pa_plan_t* plan, const void* q, const void* k_po
   a.table_stride = 0;
   a.seq_lens = nullptr;
   a.q_tma = q_tma ? 1 : 0;
+  a.k_atoms = k_atoms ? 1 : 0;
   a.rows_per_block = per * kTileRows;
   // Kernel parameter of 8 KB, copied into the launch: kept off the stack of callers with small
   // stacks, one per thread (the launch has taken its copy when this function returns).
@@ -1501,8 +1507,10 @@ extern "C" int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens,
   const int k_rows = per == 2 ? std::min(PS, 64) : PS;
   const int v_rows = per == 2 ? std::min(PS, 64) : std::min(PS, 128 / (D / 64));
   const int v_panels = per == 2 ? 2 : D / 64;
+  const bool k_atoms = per == 2 && PS == 16;  // as in pa_prefill
   CUtensorMap tk, tv, tq;
-  if (!make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows) ||
+  if (!(k_atoms ? make_v_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, 8, D / 64)
+                : make_k_map(&tk, k_pool, bf16, D, plan->n_kv_heads, rows, k_rows)) ||
       !make_v_map(&tv, v_pool, bf16, D, plan->n_kv_heads, rows, v_rows, v_panels))
     return PA_ERR_CUDA;
   const bool q_tma = per == 2 && kTileRows % plan->group == 0;
@@ -1534,6 +1542,7 @@ extern "C" int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens,
   a.balanced = 1;
   a.rows_per_block = per * kTileRows;
   a.q_tma = q_tma ? 1 : 0;
+  a.k_atoms = k_atoms ? 1 : 0;
   a.batch = plan->batch;
   a.table_stride = table_stride;
   thread_local ItemTable table;

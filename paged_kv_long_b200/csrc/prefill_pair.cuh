@@ -479,20 +479,36 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       return r_ok;
     };
     uint32_t issued = 0;  // fills this warp issued
-    // K half tile m (keys 64*rank..+63 of tile m, all of D): slot k holds panels 2k, 2k+1
+    // K half tile m (keys 64*rank..+63 of tile m, all of D) in two slots. Per-panel boxes: slot
+    // k holds panels 2k, 2k+1 (64 keys each). Atom boxes (a.k_atoms): box i = keys 8i..8i+7 x
+    // all four panels (4 KB, panel after panel) at 4 KB * i from the first slot, boxes 4k..4k+3
+    // in slot k; the half tile's two slots are adjacent (KSLOT is even).
     auto issue_k = [&](int m, int32_t rows) {
       for (int k = 0; k < 2 && ok; ++k) {
         const uint32_t q = 2u * (uint32_t)m + (uint32_t)k;
-        const int l = lane, pl = l / k_per_panel, sub = l - pl * k_per_panel;
-        const int32_t row = key_row(rows, 64 * (int)rank + sub * k_rows);
         const uint32_t sl = pair_k_slot(q);
-        if (!(ok = acquire(sl, q / C::KSLOT, false))) break;
-        if (l < 2 * k_per_panel) {
-          const uint32_t dst = slot_addr(sl) + pl * (kPanel / 2) + sub * k_rows * 128;
-          if (rank == 0)
-            tma_load_3d(dst, &tm_k, bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
-          else
-            tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
+        if (a.k_atoms) {
+          const int32_t row = key_row(rows, 64 * (int)rank + 8 * (4 * k + (lane & 3)));
+          if (!(ok = acquire(sl, q / C::KSLOT, false))) break;
+          if (lane < 4) {
+            const uint32_t dst = slot_addr(sl) + (uint32_t)lane * 4096u;
+            if (rank == 0)
+              tma_load_4d(dst, &tm_k, bar(C::B_FULL + sl), 0, row, 0, g);
+            else
+              tma_load_4d_pair(dst, &tm_k, leader_bar(C::B_FULL + sl), 0, row, 0, g);
+          }
+        } else {
+          const int l = lane, pl = l / k_per_panel, sub = l - pl * k_per_panel;
+          const int32_t row = key_row(rows, 64 * (int)rank + sub * k_rows);
+          if (!(ok = acquire(sl, q / C::KSLOT, false))) break;
+          if (l < 2 * k_per_panel) {
+            const uint32_t dst = slot_addr(sl) + pl * (kPanel / 2) + sub * k_rows * 128;
+            if (rank == 0)
+              tma_load_3d(dst, &tm_k, bar(C::B_FULL + sl), (2 * k + pl) * 64, g, row);
+            else
+              tma_load_3d_pair(dst, &tm_k, leader_bar(C::B_FULL + sl), (2 * k + pl) * 64, g,
+                               row);
+          }
         }
         issued = q + 1;
       }
@@ -574,10 +590,33 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // S(m) = Q K(m)^T into the S buffer once the softmax has read S(m-1): slot k of the K
         // half tile holds D panels 2k and 2k+1 (Q panels 2k, 2k+1). S(m) is completion m of
         // s_full and the read of S(m) arrival m of s_free.
+        // Atom boxes: panel p of the half tile starts 1 KB * p into its first slot, its 8-key
+        // atoms 4 KB apart across both slots, which are waited for first and released after
+        // all four panels.
+        const uint64_t k_desc_atoms = smem_desc_sw128(sb + C::RING_OFF, 16, 4096);
         ok = wait_cluster(bar(C::B_QFULL), 0);
         for (int m = 0; m < n && ok; ++m) {
           if (m >= 1) ok = wait_cluster(bar(C::B_SFREE), (uint32_t)(m - 1) & 1u);
           const uint32_t q0 = 2u * (uint32_t)m;
+          if (a.k_atoms) {
+            const uint32_t sl0 = pair_k_slot(q0), sl1 = pair_k_slot(q0 + 1);
+            if (ok) ok = wait_fill(sl0, pair_k_phase(q0));
+            if (ok) ok = wait_fill(sl1, pair_k_phase(q0 + 1));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const uint64_t ad = q_desc + p * kSlotDesc;
+              const uint64_t bd = k_desc_atoms + sl0 * kSlotDesc + p * (1024 >> 4);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                umma_ss_pair(s_tmem, ad + 2 * ks, bd + 2 * ks, idesc_qk, (p | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(bar(C::B_EMPTY + sl0), kBoth);
+            umma_commit_pair(bar(C::B_EMPTY + sl1), kBoth);
+            umma_commit_pair(bar(C::B_SFULL), kBoth);
+            continue;
+          }
 #pragma unroll
           for (int k = 0; k < 2 && ok; ++k) {
             if (!(ok = wait_fill(pair_k_slot(q0 + k), pair_k_phase(q0 + k)))) break;
