@@ -775,10 +775,14 @@ def gpu_arm(args):
     # ---- prefill kernel roofline: algorithmic FLOPs over its summed launch durations
     kern_total_ms = sum(sum(k) for k in kern_ms) / len(kern_ms)
     kern_tflops = flops / (kern_total_ms / 1e3) / 1e12
-    # The prefill kernel is timed inside back-to-back steps of the whole prefill (tens of
-    # milliseconds of dense tensor work without a pause), which run under the power cap after
-    # the first few steps: its denominator is the measured sustained (power-capped) GEMM rate.
-    peak = peaks["bf16_tflops_sustained"]
+    # Denominator: the measured burst GEMM rate for a kernel that runs at full clock, the
+    # sustained (power-capped) one for a kernel timed inside back-to-back steps long enough to
+    # reach the power cap, read from the timed window's clocks: median SM clock below 95 % of
+    # its maximum with sw_power_cap active (c5's 20 steps: ~7 ms each, capped after ~4 steps).
+    power_capped = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+                        and "sw_power_cap" in clocks.get("reasons", [])
+                        and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    peak = peaks["bf16_tflops_sustained"] if power_capped else peaks["bf16_tflops"]
     t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
 
     traffic, traffic_note = None, "no capture of this kernel build"
@@ -889,12 +893,16 @@ def gpu_arm(args):
                      "unit": "TFLOP/s", "frac": kern_tflops / peak, "traffic": traffic,
                      "traffic_source": traffic_note,
                      "peak_source": (f"{peaks['source']} bf16 dense, sustained (seconds of "
-                                     "back-to-back GEMMs under the power cap): the kernel is "
-                                     f"timed inside {args.steps} back-to-back steps, whose clock "
-                                     "drops under the power cap (see clocks)"),
+                                     "back-to-back GEMMs under the power cap): the timed steps "
+                                     "ran power-capped (clocks: median SM clock below 95 % of "
+                                     "max, sw_power_cap)" if power_capped else
+                                     f"{peaks['source']} bf16 dense, burst: the timed steps ran "
+                                     "at full clock"),
                      # the same kernel against the measured burst GEMM rate (full clock)
                      "frac_of_burst_peak": kern_tflops / peaks["bf16_tflops"],
+                     "frac_of_sustained_peak": kern_tflops / peaks["bf16_tflops_sustained"],
                      "burst_peak": peaks["bf16_tflops"],
+                     "sustained_peak": peaks["bf16_tflops_sustained"],
                      "kernel_ms_each_step": [round(sum(k), 4) for k in kern_ms],
                      "step_frac_of_roofline": t_roof / (t_step / 1e3),
                      # the step split: the prefill launches' summed event time, and the rest

@@ -1642,7 +1642,8 @@ extern "C" int pa_kv_append(int n_kv_heads, int head_dim, int page_size, int dty
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
     return PA_ERR_INVALID_ARG;
   const int row_vecs = n_kv_heads * head_dim * 2 / 16;
-  const int64_t warps = chunk_rows;  // one per position (its K and V rows)
+  const int64_t pieces = (int64_t)chunk_rows * row_vecs;  // 16-byte pieces per tensor
+  const int64_t warps = (pieces + 32 * kAppendBatch - 1) / (32 * kAppendBatch);
   const int64_t blocks = (warps + 7) / 8;
   if (blocks >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   kv_append_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
