@@ -185,8 +185,9 @@ int pa_combine(const pa_plan_t* plan, const float* lse_ws, uint64_t ws_bytes, fl
  * each (its own K/V already in the pool), every key of the sequence visible. Fills a plan whose
  * chunk_rows = batch (one row per sequence), q_tiles = 1 (needs G <= 128), batch = batch and
  * splits S: the history of every sequence is cut into S splits so that batch * Hkv * S units
- * fill num_sms SMs (about two per SM, at most 32 and at most the 128-key tiles of
- * max_seq_len), or exactly splits_override. ws_bytes = S * batch * Hq * (D + 1) * 4 when S > 1,
+ * fill the CTA slots (about two units per slot, at most 32 and at most the 128-key tiles of
+ * max_seq_len), or exactly splits_override. A slot is an SM, or half an SM when the group
+ * G <= 8 and D is 128 or 256 (those steps run two CTAs per SM; see pa_decode). ws_bytes = S * batch * Hq * (D + 1) * 4 when S > 1,
  * in the layout of pa_prefill's split workspace with batch in place of R, so pa_combine
  * merges it. Returns PA_OK, PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED. Pure host code.
  * Source: generation over a long cache, where every new token reads its sequence's whole
@@ -199,7 +200,9 @@ int pa_decode_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int
                    pa_plan_t* plan);
 
 /*
- * pa_decode — batched paged decode attention on `stream` (single-CTA kernel at every head dim).
+ * pa_decode — batched paged decode attention on `stream`. With G <= 8 at head dim 128 or 256 the
+ * keys take the tensor cores' M side (S^T = K Q^T, O^T = V^T P^T, two CTAs per SM); otherwise
+ * the single-CTA prefill kernel runs one 128-row Q tile per unit.
  *   q            device [batch][Hq][D] of dtype: the new token of each sequence.
  *   k_pool,v_pool device [num_pages][PS][Hkv][D], 16-byte aligned.
  *   block_table  device int32 [batch][table_stride]: sequence b's logical page -> physical page.
