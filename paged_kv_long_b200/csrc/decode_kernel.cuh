@@ -68,10 +68,13 @@ __device__ __forceinline__ uint16_t to16(float x) {
     return __half_as_ushort(__float2half_rn(x));
 }
 
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
-    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const PrefillArgs a_in) {
+// BAL: block b runs work item b of a balanced one-row batch (the item's sequence, KV head and
+// key range; an uncut row block writes the output, a part of a cut one its partial and LSE in
+// the item's workspace slot, merged by combine_blocks_kernel). Otherwise block b is decode unit
+// b of pa_decode (device lengths, uniform splits).
+template <int D, bool BF16, bool BAL>
+__device__ __forceinline__ void decode_body(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                            const PrefillArgs& a_in, const ItemTable* items) {
   PrefillArgs a = a_in;
   using C = DecCfg<D>;
   constexpr int NP = C::NP, NSLOT = C::NSLOT, NH = D / 128;  // NH: 128-dim halves of O^T
@@ -81,9 +84,19 @@ __global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  int g, s;
+  int g, s = 0, slot = kSlotUniform;
   int64_t kt0, kt1;
-  decode_unit<D>(a, reinterpret_cast<int32_t*>(smem + C::RING_OFF), &g, &s, &kt0, &kt1);
+  if constexpr (BAL) {
+    const PaItem it = items->item[blockIdx.x];
+    const int32_t rb = batch_rebase<D>(a, *items, it.rb);  // one Q tile per sequence: g = rb
+    int64_t qt;
+    rb_coords(rb, a.q_tiles, a.Hkv, &qt, &g);
+    kt0 = it.kt0;
+    kt1 = it.kt1;
+    slot = it.slot;
+  } else {
+    decode_unit<D>(a, reinterpret_cast<int32_t*>(smem + C::RING_OFF), &g, &s, &kt0, &kt1);
+  }
   const int n = (int)(kt1 - kt0);
   if (n == 0) {
     empty_unit<D>(a, 0, g, s);
@@ -293,8 +306,17 @@ __global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
         ls[h] = (sums[h] + sums[8 + h]) + (sums[16 + h] + sums[24 + h]);
         inv_l[h] = ls[h] > 0.f ? 1.f / ls[h] : 0.f;
       }
-      const bool partial = a.splits > 1;
-      const int64_t row0 = partial ? (int64_t)s * a.ws_split_rows + g * G : (int64_t)g * G;
+      // Destination rows of heads g*G + h: the output, a uniform split's partial, or the packed
+      // rows h of a balanced item's workspace slot.
+      bool partial;
+      int64_t row0;
+      if (slot >= 0) {
+        partial = true;
+        row0 = (int64_t)slot * a.rows_per_block;
+      } else {
+        partial = slot == kSlotUniform && a.splits > 1;
+        row0 = partial ? (int64_t)s * a.ws_split_rows + g * G : (int64_t)g * G;
+      }
       float* base = partial ? a.ws_o : a.out;
 #pragma unroll
       for (int hf = 0; hf < NH; ++hf) {
@@ -404,4 +426,19 @@ __global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
     tc_fence_after();
     tmem_dealloc(tmem, kDecTmemCols);
   }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const PrefillArgs a) {
+  decode_body<D, BF16, false>(tm_k, tm_v, a, nullptr);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, kDecCtasPerSm)
+    decode_batch_kernel(const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a,
+                        const __grid_constant__ ItemTable items) {
+  decode_body<D, BF16, true>(tm_k, tm_v, a, &items);
 }

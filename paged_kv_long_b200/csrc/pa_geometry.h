@@ -94,6 +94,15 @@ constexpr int kMaxSplitBlocks = 256;
 struct PaSeq {
   int32_t q_row0, rows, hist, rb0;
 };
+// Batches run on the swapped decode kernel too when every sequence has at most one query row (a
+// decode step with host-side lengths) and their row blocks are single CTAs.
+inline bool batch_decode_swapped(int D, int G, int per, const PaSeq* seq, int n) {
+  if (per != 1 || !decode_swapped(D, G)) return false;
+  for (int b = 0; b < n; ++b)
+    if (seq[b].rows > 1) return false;
+  return true;
+}
+
 constexpr int kMaxSeqs = 256;
 
 // The sequence that owns global row block rb: the last b with seq[b].rb0 <= rb (rb0 ascending).

@@ -1177,26 +1177,50 @@ cudaError_t launch_d(bool paged, bool bf16, int64_t grid, cudaStream_t st, const
               : launch_prefill<D, false, false>(grid, st, tk, tv, a, it);
 }
 
-template <int D, bool BF16>
-cudaError_t launch_decode(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
-                          const CUtensorMap& tv, const PrefillArgs& a) {
-  auto kern = decode_kernel<D, BF16>;
-  static std::atomic<uint64_t> configured{0};  // one bit per device ordinal
+// The decode kernels' attributes (shared memory, carveout for two CTAs per SM), once per device.
+template <class K>
+cudaError_t configure_decode(K kern, int smem, std::atomic<uint64_t>& configured) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DecCfg<D>::LAUNCH_SMEM);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  kern<<<(unsigned)grid, kThreads, DecCfg<D>::LAUNCH_SMEM, st>>>(tk, tv, a);
+  return cudaSuccess;
+}
+
+template <int D, bool BF16, bool BAL>
+cudaError_t launch_decode(int64_t grid, cudaStream_t st, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const PrefillArgs& a, const ItemTable& it) {
+  static std::atomic<uint64_t> configured{0};  // one bit per device ordinal
+  cudaError_t e;
+  if constexpr (BAL) {
+    e = configure_decode(decode_batch_kernel<D, BF16>, DecCfg<D>::LAUNCH_SMEM, configured);
+    if (e != cudaSuccess) return e;
+    decode_batch_kernel<D, BF16><<<(unsigned)grid, kThreads, DecCfg<D>::LAUNCH_SMEM, st>>>(
+        tk, tv, a, it);
+  } else {
+    e = configure_decode(decode_kernel<D, BF16>, DecCfg<D>::LAUNCH_SMEM, configured);
+    if (e != cudaSuccess) return e;
+    decode_kernel<D, BF16><<<(unsigned)grid, kThreads, DecCfg<D>::LAUNCH_SMEM, st>>>(tk, tv, a);
+  }
   return cudaGetLastError();
+}
+
+template <bool BAL>
+cudaError_t launch_decode_d(int D, bool bf16, int64_t grid, cudaStream_t st,
+                            const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
+                            const ItemTable& it) {
+  return D == 128 ? (bf16 ? launch_decode<128, true, BAL>(grid, st, tk, tv, a, it)
+                          : launch_decode<128, false, BAL>(grid, st, tk, tv, a, it))
+                  : (bf16 ? launch_decode<256, true, BAL>(grid, st, tk, tv, a, it)
+                          : launch_decode<256, false, BAL>(grid, st, tk, tv, a, it));
 }
 
 // Paged single-CTA launches of decode and batches (sq: every Q tile holds <= 8 packed rows).
@@ -1408,10 +1432,7 @@ extern "C" int pa_decode(const pa_plan_t* plan, const void* q, const void* k_poo
   if (grid >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   cudaError_t e;
   if (decode_swapped(D, plan->group))
-    e = D == 128 ? (bf16 ? launch_decode<128, true>(grid, st, tk, tv, a)
-                         : launch_decode<128, false>(grid, st, tk, tv, a))
-                 : (bf16 ? launch_decode<256, true>(grid, st, tk, tv, a)
-                         : launch_decode<256, false>(grid, st, tk, tv, a));
+    e = launch_decode_d<false>(D, bf16, grid, st, tk, tv, a, table);
   else
     e = launch_paged_single(D, bf16, plan->group <= 8, grid, st, tk, tv, a, table);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -1557,6 +1578,8 @@ extern "C" int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens,
   if (per == 2)
     e = bf16 ? launch_pair<true, true>(grid, cs, tk, tv, tq, a, table)
              : launch_pair<true, false>(grid, cs, tk, tv, tq, a, table);
+  else if (batch_decode_swapped(D, plan->group, per, bt.seq.data(), (int)bt.seq.size()))
+    e = launch_decode_d<true>(D, bf16, grid, cs, tk, tv, a, table);
   else
     e = launch_paged_single(D, bf16, small_q, grid, cs, tk, tv, a, table);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -347,6 +347,9 @@ int batch_ctas_per_unit(int head_dim, int G, int batch, const int32_t* q_lens) {
 
 bool build_batch(int num_sms, int head_dim, int per, int G, int Hkv, const Batch& bt,
                  Schedule* out) {
+  // One-row batches on the swapped decode kernel: two CTA slots per SM.
+  if (batch_decode_swapped(head_dim, G, per, bt.seq.data(), (int)bt.seq.size()))
+    num_sms *= kDecCtasPerSm;
   // one sequence: the single piece's schedule (row blocks numbered the same way)
   if (bt.seq.size() == 1 && per == ctas_per_unit_for(head_dim))
     return balanced_piece(q_tiles_for(bt.seq[0].rows, G), bt.seq[0].rows, bt.seq[0].hist, G,

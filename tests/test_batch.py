@@ -351,3 +351,18 @@ def test_gpu_batched_decode_matches_uniform_decode_and_oracle():
     torch.cuda.synchronize()
     U.assert_close(dec.cpu().numpy(), ref, "uniform decode")
     assert bd.device_error(reset=True)[0] == 0
+
+
+def test_one_row_batches_plan_two_cta_slots_per_sm():
+    """One-row batches with G <= 8 at head dim 128 / 256 run the swapped-operand decode kernel,
+    two CTAs per SM: their items are cut for 2 x num_sms workers (each worker's share ends at a
+    cut, so there are at least that many items); other batches keep one worker per SM."""
+    bd = _bd()
+    B, hist = 32, np.full(32, 20000)
+    ones = np.ones(B, dtype=np.int32)
+    for D in (128, 256):
+        bp = bd.batch_plan(16, 2, D, 16, ones, hist, "bf16", num_sms=148)
+        assert bp.plan.ctas_per_unit == 1 and bp.plan.units >= 2 * 148
+    for Hq, D, q_lens in ((32, 256, ones), (16, 64, ones), (16, 256, 2 * ones)):
+        bp = bd.batch_plan(Hq, 2, D, 16, q_lens, hist, "bf16", num_sms=148)
+        assert bp.plan.units < 2 * 148
