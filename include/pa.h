@@ -259,6 +259,9 @@ int pa_batch_plan(int num_sms, int n_q_heads, int n_kv_heads, int head_dim, int 
  *   lse_ws       workspace of plan->ws_bytes when ws_bytes > 0; then call pa_batch_combine.
  * Returns PA_OK, PA_ERR_INVALID_ARG (arrays that do not rebuild the plan's schedule, or a
  * plan that is not a batch plan), PA_ERR_WORKSPACE or PA_ERR_CUDA.
+ * A batch in which every sequence has at most one query row, with G <= 8 at head dim 128 or
+ * 256, runs on pa_decode's kernel (keys on the tensor cores' M side, two CTAs per SM), and
+ * pa_batch_plan cuts its items for two CTA slots per SM.
  */
 int pa_batch_prefill(const pa_plan_t* plan, const int32_t* q_lens, const int64_t* hist_lens,
                      const void* q, const void* k_pool, const void* v_pool,
