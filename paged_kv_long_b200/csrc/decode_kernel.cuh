@@ -1,5 +1,6 @@
-// decode_kernel.cuh — one decode step (one query token per sequence, device-side lengths) with
-// the operands of both products swapped. Included by pa_kernels.cu.
+// decode_kernel.cuh — one decode step (one query token per sequence: pa_decode with device-side
+// lengths, or a one-row batch with host-side lengths) with the operands of both products
+// swapped. Included by pa_kernels.cu.
 //
 // A decode unit (sequence, KV head, split) has G <= 8 query rows, so a 128-row Q tile is almost
 // all padding. Here the keys take the MMA's M side instead:
@@ -110,7 +111,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tm_k, const CUten
     pre_row1 = tile_page_row<true>(a, kt0, n, 1, lane, report);
   }
   auto bar = [&](int i) -> uint32_t { return sb + C::BAR_OFF + 8u * (uint32_t)i; };
-  auto slot_addr = [&](uint32_t slot) -> uint32_t { return sb + C::RING_OFF + slot * kPanel; };
+  auto slot_addr = [&](uint32_t r) -> uint32_t { return sb + C::RING_OFF + r * kPanel; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF + 4);
 
