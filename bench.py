@@ -37,9 +37,9 @@ L2_FLUSH_BYTES = 512 << 20
 # sources hash to `sources`; after any change to them the bench reports null until the
 # captures are taken again.
 TRAFFIC_CAPTURE = {
-    "workload": "c5", "sources": "2afb64ec921027e1", "bytes_per_launch": 110.18e6,
+    "workload": "c5", "sources": "fa8f8d4e9d5b6d04", "bytes_per_launch": 108.12e6,
     "how": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch each of chunks 0, 3, "
-            "6, 9, 12 and 15 (21.1, 39.8, 65.9, 94.7, 157.8, 323.2 MB; three launches per capture "
+            "6, 9, 12 and 15 (21.2, 39.3, 65.0, 94.2, 149.9, 321.2 MB; three launches per capture "
             "of bench.py --section piece), linear in between, mean over the 16 chunks")}
 
 
