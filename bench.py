@@ -74,6 +74,19 @@ def load_peaks():
                     source="fallback")
 
 
+def roofline_peak(clocks: dict, peaks: dict) -> tuple[float, bool]:
+    """The bf16 denominator of an in-step kernel and whether the timed steps ran power-capped.
+    The measured burst GEMM rate applies to a kernel that runs at full clock, the sustained
+    (power-capped) one to a kernel timed inside back-to-back steps long enough to reach the power
+    cap, read from the timed window's clocks: median SM clock below 95 % of its maximum with
+    sw_power_cap active (c5's 20 steps: ~7 ms each, capped after ~4 steps). Without clock
+    samples the burst figure (the stricter one) applies."""
+    capped = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+                  and "sw_power_cap" in clocks.get("reasons", [])
+                  and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    return (peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]), capped
+
+
 class ClockSampler:
     """Clocks and throttle reasons while running: nvidia-smi every 20 ms (the sampler is given a
     moment to start before the timed region) and, where NVML is importable, the SM clock, power
@@ -775,14 +788,7 @@ def gpu_arm(args):
     # ---- prefill kernel roofline: algorithmic FLOPs over its summed launch durations
     kern_total_ms = sum(sum(k) for k in kern_ms) / len(kern_ms)
     kern_tflops = flops / (kern_total_ms / 1e3) / 1e12
-    # Denominator: the measured burst GEMM rate for a kernel that runs at full clock, the
-    # sustained (power-capped) one for a kernel timed inside back-to-back steps long enough to
-    # reach the power cap, read from the timed window's clocks: median SM clock below 95 % of
-    # its maximum with sw_power_cap active (c5's 20 steps: ~7 ms each, capped after ~4 steps).
-    power_capped = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
-                        and "sw_power_cap" in clocks.get("reasons", [])
-                        and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
-    peak = peaks["bf16_tflops_sustained"] if power_capped else peaks["bf16_tflops"]
+    peak, power_capped = roofline_peak(clocks, peaks)
     t_roof = max(flops / (peak * 1e12), wl.kv_bytes() / (peaks["hbm_gbs"] * 1e9))
 
     traffic, traffic_note = None, "no capture of this kernel build"

@@ -52,3 +52,17 @@ def test_traffic_capture_is_keyed_to_the_kernel_sources():
     assert len(h) == 16 and int(h, 16) >= 0
     cap = bench.TRAFFIC_CAPTURE
     assert cap is None or set(cap) == {"workload", "sources", "bytes_per_launch", "how"}
+
+
+def test_roofline_peak_follows_the_timed_window_clocks():
+    """Burst peak at full clock; sustained only when the timed steps ran power-capped (median SM
+    clock below 95 % of max with sw_power_cap); burst when the clock record is missing."""
+    peaks = {"bf16_tflops": 1642.9, "bf16_tflops_sustained": 1392.3}
+    capped = {"sm_mhz": 1507, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.roofline_peak(capped, peaks) == (1392.3, True)
+    full = {"sm_mhz": 1965, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.roofline_peak(full, peaks) == (1642.9, False)
+    low_no_reason = {"sm_mhz": 1500, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.roofline_peak(low_no_reason, peaks) == (1642.9, False)
+    missing = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+    assert bench.roofline_peak(missing, peaks) == (1642.9, False)
