@@ -255,6 +255,12 @@ CASES = [
     ("d128_empty_seq", [100, 5, 2000], [64, 0, 333], 32, 8, 128, 32, "bf16", None),
     ("d128_cuts", [3000, 50, 7000], [128, 300, 40], 8, 1, 128, 16, "f16", 5),
     ("d64_g16", [0, 900], [300, 77], 32, 2, 64, 128, "f16", 4),
+    # one-row batches on the swapped-operand decode kernel (G <= 8 at head dim 128 / 256): empty
+    # sequences, one key, page and tile edges, and few SMs so that items are cut and merged
+    ("d128_one_row_swapped", [0, 15, 16, 127, 128, 4000, 9000, 0], [1, 1, 1, 1, 1, 1, 1, 0],
+     16, 4, 128, 16, "bf16", 12),
+    ("d256_one_row_g1_swapped", [3000, 1, 511], [1, 1, 1], 2, 2, 256, 32, "f16", 4),
+    ("d256_one_row_ps128_swapped", [10000, 300, 64], [1, 1, 1], 16, 2, 256, 128, "bf16", 8),
 ]
 
 
