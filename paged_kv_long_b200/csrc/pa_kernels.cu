@@ -2,7 +2,7 @@
 //
 // prefill_kernel: one CTA per unit — (KV head, packed Q tile, history split) for uniform splits,
 //   a work item (a run of a row block's KV tiles) for balanced plans, (sequence, KV head, split)
-//   for batched decode.
+//   for batched decode whose group the swapped decode kernel does not take.
 //   The operation is prefill attention of a query chunk against a long history read through
 //   a paged KV cache (BaseRT issue #51, "Results"), with the history of a piece cut into
 //   splits whose partials a reduce merges (splash PR #33, "What changed"). The B200 design:
@@ -20,6 +20,8 @@
 //   Every wait is bounded: on expiry the kernel sets the timeout bit, abandons its work,
 //   waits for its own copies and MMAs in flight, frees tensor memory and exits.
 // prefill_pair_kernel (prefill_pair.cuh): head dim 256 on CTA pairs (cta_group::2, M = 256).
+// decode_kernel, decode_batch_kernel (decode_kernel.cuh): one query token per sequence with the
+//   keys on the MMA's M side (S^T = K Q^T, O^T = V^T P^T), two CTAs per SM.
 // combine_kernel: one warp per (row, head) merges the S partials with a log-sum-exp
 //   weighting (the "reduce" of splash PR #33); combine_blocks_kernel does the same for the
 //   cut row blocks of balanced plans.
